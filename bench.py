@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 RAM-Net layer core.
+
+One step = one ``ramnet_scan_forward`` call (address decode of keys and queries, CAPE,
+Gated Sparse Update, sparse read, RMSNorm, gate) over the 340M-like Top-8 prefill
+workload: B=8 sequences x T=4096 tokens x H=8 heads, d_p=4, U=5 (M=1024 slots), K=8,
+d_v=128, bf16 inputs and output, fp32 slot state, zero initial state.  Inputs are
+resident in HBM when timing starts; L2 is flushed (256 MiB write) between timed steps.
+
+The JSON line also carries:
+  roofline     algorithmic bytes of the step / device time, against the measured HBM copy
+               bandwidth (MEASURED_PEAKS.json);
+  e2e          the same metric through the public API with pinned host buffers (H2D of the
+               step's inputs and D2H of y inside the timed region);
+  decode       the batched decode step (B=256, H=16, M=4096, K=16, d_v=128, state resident
+               in HBM), 1024 consecutive steps replayed from one CUDA graph;
+  cpu_baseline the CPU oracle on a bounded sample of the same workload (rank 0, N=1 only).
+
+``--impl reference`` times the CPU oracle itself (the reference arm: there is no
+reference implementation to install; the pages ship no code).
+
+Multi-GPU (torchrun): every (b,h) head is independent, so each rank runs its own full
+batch with no data-path collective (weak scaling); NCCL is used only for the barrier and
+the max-over-ranks of the step time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_slot_recurrent_b200.workloads import WORKLOADS, generate  # noqa: E402
+
+METRIC = "RAM-Net layer tokens/s (prefill scan, decode step) and % of HBM roofline"
+PREFILL = "prefill_340m_top8"
+DECODE = "decode_b256"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ accounting
+
+def prefill_algorithmic_bytes(w, in_bytes=2, out_bytes=2, state_in=False) -> int:
+    """Bytes a step must move at least: per token-head the two address logit vectors, v,
+    g, z and y; per head the final state (S fp32 [M,d_v] + m fp32 [M]); the zero initial
+    state is not read."""
+    per_th = 2 * w.L * in_bytes + w.d_v * in_bytes + in_bytes + w.d_v * in_bytes + w.d_v * out_bytes
+    per_head = w.M * w.d_v * 4 + w.M * 4
+    n_th = w.B * w.T * w.H
+    return n_th * per_th + w.B * w.H * per_head * (2 if state_in else 1)
+
+
+def decode_algorithmic_bytes(w, in_bytes=2, out_bytes=2) -> int:
+    """Per (b,h) per step: inputs and y, the K write rows read and written, the K read rows
+    read, and the K masses read and written (fp32)."""
+    per_unit = 2 * w.L * in_bytes + w.d_v * in_bytes + in_bytes + w.d_v * in_bytes + w.d_v * out_bytes
+    per_unit += w.K * w.d_v * 4 * 3 + w.K * 4 * 2
+    return w.B * w.H * per_unit
+
+
+def state_elements_per_step(K: int, d_v: int, heads: int) -> int:
+    """State elements a decode step touches: K read rows + K write rows per head."""
+    return heads * 2 * K * d_v
+
+
+# ------------------------------------------------------------------ environment helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_slot_recurrent_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu capture, only if the kernel sources are
+    unchanged since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel]
+        if e.get("source_hash") == kernel_source_hash():
+            return e
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda") if torch.cuda.is_available() else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank processed tokens_per_rank in at most max_ms."""
+    return world * tokens_per_rank / (max_ms / 1e3)
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+
+def oracle_sample(w, n_heads: int, threads: int):
+    """Run the CPU oracle on the first n_heads (b,h) heads (whole sequences) of the
+    workload; returns (seconds, token-heads processed)."""
+    import oracle
+    oracle.build()
+    nb = max(1, (n_heads + w.H - 1) // w.H)
+    sub = w.with_(B=nb)
+    inp = generate(sub, seed=0)
+    ocfg = oracle.OracleConfig(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
+    t0 = time.perf_counter()
+    oracle.scan_forward(ocfg, inp["k_logits"], inp["q_logits"], inp["v"], inp["g"], inp["z"],
+                        cape_mask=inp["cape_mask"], pos0=inp["pos0"], nthreads=threads)
+    return time.perf_counter() - t0, nb * w.H * w.T
+
+
+def cpu_baseline(w, cores: int):
+    n_heads = min(w.B * w.H, max(8, 2 * cores))
+    secs, th = oracle_sample(w, n_heads, cores)
+    heads = ((n_heads + w.H - 1) // w.H) * w.H
+    return {"value": th / w.H / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} (b,h) heads x T={w.T} tokens of {w.name} (tokens/s = token-heads/s / H)",
+            "seconds": round(secs, 3)}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    w = WORKLOADS[PREFILL]
+    cores = os.cpu_count() or 1
+    n_heads = min(w.B * w.H, cores)
+    for _ in range(args.warmup):
+        oracle_sample(w, n_heads, cores)
+    secs = []
+    th = 0
+    for _ in range(args.steps):
+        s, th = oracle_sample(w, n_heads, cores)
+        secs.append(s)
+    ms = 1e3 * statistics.mean(secs)
+    value = th / w.H / (ms / 1e3)
+    heads = ((n_heads + w.H - 1) // w.H) * w.H
+    sample = f"{heads} (b,h) heads x T={w.T} tokens of {w.name} per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_p": w.d_p, "U": w.U, "M": w.M, "K": w.K,
+            "d_v": w.d_v, "in_dtype": "bf16", "out_dtype": "bf16", "state": "fp32", "cape": w.cape,
+            "l2": "flushed between timed steps (256 MiB write)",
+            "parallelism": f"dp{world} (independent heads per rank, no collective)"}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, world, rank, local):
+    from sparse_slot_recurrent_b200 import ramnet
+    ramnet.load()
+    w = WORKLOADS[PREFILL]
+    cfg = ramnet.Config(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
+    dev = torch.device("cuda", local)
+    inp = generate(w, seed=rank)
+    host = {k: v.pin_memory() for k, v in inp.items() if torch.is_tensor(v)}
+    d = {k: v.to(dev) for k, v in host.items()}
+    y = torch.empty((w.B, w.T, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((w.B, w.H, w.M, w.d_v), dtype=torch.float32, device=dev)
+    m = torch.empty((w.B, w.H, w.M), dtype=torch.float32, device=dev)
+    ws = torch.empty(ramnet.scan_workspace_bytes(cfg, w.B, w.T, w.H), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"], cape_mask=d["cape_mask"],
+                            pos0=d["pos0"], y=y, S_out=S, m_out=m, workspace=ws, stream=stream)
+
+    launches_per_step = 3  # key decode, query decode, scan
+    for _ in range(args.warmup):
+        step()
+    ramnet.sync_status(stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    clk = clocks.stop()
+    ramnet.sync_status(stream)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_max = dist_max(ms, world)
+    tokens = w.B * w.T
+    value = weak_scaling_value(tokens, world, ms_max)
+
+    # roofline of the timed step against measured HBM bandwidth
+    peak, peak_kind = measured_peaks()
+    alg = prefill_algorithmic_bytes(w)
+    achieved = alg / (ms / 1e3) / 1e9
+    traffic = recorded_traffic("scan_forward")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                "kernel": "ramnet_scan_forward (decode_addresses x2 + scan_tmem)",
+                "algorithmic_bytes": alg, "peak_kind": f"{peak_kind} hbm_gbs"}
+
+    # end to end through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        keys = ("k_logits", "q_logits", "v", "g", "z", "cape_mask", "pos0")
+        yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        d2h = yh.numel() * yh.element_size()
+
+        def e2e_step():
+            for k in keys:
+                d[k].copy_(host[k], non_blocking=True)
+            step()
+            yh.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        dist_barrier(world)
+        for i in range(args.steps):
+            flush.zero_()
+            ee[i][0].record(stream)
+            e2e_step()
+            ee[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = dist_max(statistics.mean(a.elapsed_time(b) for a, b in ee), world)
+        e2e = {"value": weak_scaling_value(tokens, world, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    decode = None if args.no_decode else run_decode(args, world, local)
+    del flush
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; shapes of the 340M-like layer)",
+                "config": config_of(w, world), "roofline": roofline, "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps, "clocks": clk, "decode": decode}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, os.cpu_count() or 1)
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, world, local):
+    """1024 consecutive decode steps of the batched workload, one CUDA graph."""
+    from sparse_slot_recurrent_b200 import ramnet
+    w = WORKLOADS[DECODE]
+    cfg = ramnet.Config(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
+    dev = torch.device("cuda", local)
+    inp = generate(w, seed=0)
+    ring = [{k: inp[k][:, r].contiguous().to(dev) for k in ("k_logits", "q_logits", "v", "g", "z")}
+            for r in range(w.ring)]
+    mask = inp["cape_mask"].to(dev)
+    gen = torch.Generator(device=dev).manual_seed(1)
+    S = torch.randn((w.B, w.H, w.M, w.d_v), device=dev, generator=gen)
+    m = torch.rand((w.B, w.H, w.M), device=dev, generator=gen) * 1.5 + 0.5
+    pos = torch.arange(w.T, dtype=torch.int32, device=dev).view(w.T, 1).expand(w.T, w.B).contiguous()
+    y = torch.empty((w.B, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def steps():
+        for t in range(w.T):
+            r = ring[t % w.ring]
+            ramnet.decode_step(cfg, r["k_logits"], r["q_logits"], r["v"], r["g"], r["z"], S, m, pos=pos[t],
+                               cape_mask=mask, y=y, stream=stream)
+
+    with torch.cuda.stream(stream):
+        steps()  # warm-up outside the graph
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        steps()
+    reps = max(1, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    dist_barrier(world)
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+    stream.synchronize()
+    ramnet.sync_status(stream)
+    ms = dist_max(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    del graph
+    peak, peak_kind = measured_peaks()
+    alg = decode_algorithmic_bytes(w)
+    step_ms = ms / w.T
+    achieved = alg / (step_ms / 1e3) / 1e9
+    return {"workload": w.name, "steps_per_replay": w.T, "replays": reps, "B": w.B, "H": w.H, "M": w.M, "K": w.K,
+            "d_v": w.d_v, "value": weak_scaling_value(w.B * w.T, world, ms), "unit": "tokens/s",
+            "ms_per_step": step_ms, "gpu_launches_per_replay": w.T,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "k_decode_step",
+                         "algorithmic_bytes_per_step": alg, "peak_kind": f"{peak_kind} hbm_gbs"},
+            "l2": "state (8 GiB) larger than L2",
+            "state_elements_per_step": state_elements_per_step(w.K, w.d_v, w.B * w.H)}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ramnet", "reference"], default="ramnet")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    if world != args.gpus and rank == 0:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using {world}", file=sys.stderr)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("the ramnet arm needs a CUDA device")
+            run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * ramnet.h -- C ABI of the B200 (sm_100a) RAM-Net layer core.
+ *
+ * The layer follows the RAM-Net project page ("RAM-Net: Linear-Time Sequence Modeling
+ * with Sparsely Addressable State", muoncat.github.io/ramnet_web).  Each token of each
+ * head brings an address logit vector for its key (write) and its query (read), a value
+ * v, a write gate g and an output gate z.  The layer:
+ *   1. Address Decoder / Product Softmax: splits each logit vector into U groups of d_p
+ *      scores, and finds the exact Top-K of the M = d_p^U slot weights
+ *      prod_u softmax(x_u)[d_u] by a level-by-level prefix-tree search;
+ *   2. CAPE: shifts the selected slot indices cyclically by the token position on heads
+ *      whose CAPE flag is set;
+ *   3. Gated Sparse Update: updates content and write mass of the K write slots only;
+ *   4. reads the K read slots combined by their weights, applies RMSNorm over d_v and
+ *      multiplies by the output gate.
+ *
+ * Numerical definitions (identical on every entry point):
+ *   - Ranking score of one digit logit x: q(x) = round_half_even(clamp(x, -4095, 4095)
+ *     * 2^32) as a 64-bit integer (NaN ranks lowest); a slot's score is the integer sum
+ *     of its U digit scores.  Higher score wins; equal scores go to the lower slot index
+ *     (taken before the CAPE shift).  Slot index i = sum_u d_u * d_p^(U-1-u): group 0 of
+ *     the logits is the most significant digit.
+ *   - Weights of the K selected slots (rank order): renorm != 0: w_j = exp(s_j - s_0) /
+ *     sum_k exp(s_k - s_0) with s the slot's digit-logit sum; renorm == 0: w_j =
+ *     prod_u softmax(x_u)[d_u].  Logits are expected within +-4095 (the clamp also
+ *     enters the weights).
+ *   - CAPE: slot -> (slot + pos) mod M with pos = pos0[b] + t.
+ *   - Gated Sparse Update of write slot i with weight w, gate g in [0,1] (clamped):
+ *     alpha = (1 - w)^(g/(1-g)) [alpha = 1 when w == 0 or g == 0; 0 when g == 1 or
+ *     w == 1], m_i <- alpha*m_i + w, lambda = w/(m_i + eps_gsu), S_i <- S_i +
+ *     lambda*(v - S_i).  Slots not written keep content and mass bit for bit.
+ *   - Read after the token's own write: o = sum_j r_j S_{read_j};
+ *     y = o / sqrt(mean(o^2) + eps_norm) * norm_w * z.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE memory owned by the caller, unless stated otherwise; the
+ *     library never frees or keeps them.  Arrays are dense row-major (C order) with the
+ *     stated shapes; every base pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
+ *     are asynchronous on that stream: outputs are valid once the stream has reached
+ *     the call.  The caller keeps inputs alive until then.
+ *   - Argument checks happen on the host before anything is launched; a failing check
+ *     returns RAMNET_ERR_INVALID_ARG or RAMNET_ERR_UNSUPPORTED and launches nothing.
+ *     A launch error returns RAMNET_ERR_CUDA.  ramnet_last_error() describes the last
+ *     failure of the calling thread.
+ *   - Kernels that wait on other thread blocks wait a bounded number of iterations; when
+ *     a wait gives up the kernel records it in a device status word and returns early.
+ *     ramnet_sync_status() reads (and clears) that word.
+ *   - No call allocates device memory.  Scratch space comes from the caller
+ *     (ramnet_scan_forward's workspace).
+ *   - Limits: 2 <= d_p <= 16, 1 <= U <= 8, M = d_p^U <= 65536, 1 <= K <= min(M, 64),
+ *     d_v in {16, 32, 64, 128, 256}.  ramnet_scan_forward additionally needs the slot
+ *     array of one head to fit the tensor memory of at most 8 SMs (M * max(d_v,32) *
+ *     4 bytes <= 8 * 256 KiB); larger shapes return RAMNET_ERR_UNSUPPORTED.
+ */
+#ifndef RAMNET_H
+#define RAMNET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RAMNET_OK = 0,
+    RAMNET_ERR_INVALID_ARG = 1,   /* bad pointer, shape, alignment or value */
+    RAMNET_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement */
+    RAMNET_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    RAMNET_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up */
+    RAMNET_ERR_DEVICE_CHECK = 5   /* a device-side consistency check failed */
+} ramnet_status;
+
+typedef enum {
+    RAMNET_F32 = 0,
+    RAMNET_BF16 = 1
+} ramnet_dtype;
+
+/* Layer hyper-parameters.  M = d_p^U slots per head. */
+typedef struct {
+    int32_t d_p;      /* values per digit (softmax group size)            */
+    int32_t U;        /* digits per address (number of softmax groups)     */
+    int32_t K;        /* slots selected per read and per write             */
+    int32_t d_v;      /* value / slot width                                */
+    float eps_gsu;    /* epsilon of the GSU update rate (e.g. 1e-6)        */
+    float eps_norm;   /* epsilon inside the output RMSNorm (e.g. 1e-6)     */
+    int32_t renorm;   /* 1: weights renormalised over the K selected slots */
+} ramnet_config;
+
+/*
+ * ramnet_decode_addresses -- Address Decoder and CAPE for a batch of tokens.
+ * Project page: Product Softmax paragraph, the five views (exact Top-K search in the
+ * Multilevel Decision Tree view and the exactness paragraph after them), CAPE paragraphs.
+ *
+ *   logits    [B,T,H,U*d_p]  dtype `dt` (RAMNET_F32 or RAMNET_BF16)
+ *   pos0      [B] int32 start position of each sequence, or NULL (all 0)
+ *   cape_mask [H] uint8, nonzero = CAPE on for that head, or NULL (CAPE off)
+ *   idx_out   [B,T,H,K] int32: selected slot indices, best first, after CAPE
+ *   w_out     [B,T,H,K] fp32: their weights (same order)
+ * Errors: INVALID_ARG for null logits/outputs, non-positive sizes, misalignment or a
+ * config outside the limits.
+ */
+ramnet_status ramnet_decode_addresses(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                      const void* logits, ramnet_dtype dt, const int32_t* pos0,
+                                      const uint8_t* cape_mask, int32_t* idx_out, float* w_out,
+                                      void* stream);
+
+/*
+ * ramnet_scan_workspace_bytes -- scratch bytes ramnet_scan_forward needs for these sizes
+ * (the decoded addresses of both streams).  Returns 0 for invalid arguments.
+ */
+size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H);
+
+/*
+ * ramnet_scan_forward -- prefill: the whole layer core over T tokens, per (b,h) in token
+ * order.  Project page: the three-stage processing paragraph, Gated Sparse Update (four
+ * steps and the unselected-slot rule), and the GPU-execution paragraph (Top-K for all
+ * tokens in parallel first, then the recurrence).
+ *
+ *   k_logits, q_logits [B,T,H,U*d_p]  in_dt   key (write) / query (read) address logits
+ *   v, z               [B,T,H,d_v]    in_dt   value, output gate (multiplied as given)
+ *   g                  [B,T,H]        in_dt   write gate in [0,1] (activated gamma)
+ *   norm_w             [d_v] fp32 or NULL (ones)
+ *   cape_mask          [H] uint8 or NULL (off);  pos0 [B] int32 or NULL (0)
+ *   S_in               [B,H,M,d_v] fp32 initial slot contents, or NULL (zeros)
+ *   m_in               [B,H,M] fp32 initial write mass, or NULL (zeros)
+ *   y                  [B,T,H,d_v] out_dt output
+ *   S_out, m_out       final state, same shapes as S_in, m_in (may alias them)
+ *   workspace          device scratch of at least ramnet_scan_workspace_bytes() bytes,
+ *                      16-byte aligned; contents on entry are ignored
+ * Errors: INVALID_ARG (null required pointer, sizes, alignment, too small workspace),
+ * UNSUPPORTED (slot array too large for tensor memory, see limits).
+ */
+ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                  ramnet_dtype in_dt, const void* k_logits, const void* q_logits,
+                                  const void* v, const void* g, const void* z,
+                                  const float* norm_w, const uint8_t* cape_mask,
+                                  const int32_t* pos0, const float* S_in, const float* m_in,
+                                  void* y, ramnet_dtype out_dt, float* S_out, float* m_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ramnet_decode_step -- one autoregressive token per (b,h) against an HBM-resident state,
+ * touching only the slots the token selects.  Project page: GPU-execution paragraph on
+ * autoregressive decoding (no scan over the full state), plus the same three stages.
+ *
+ *   k_logits, q_logits [B,H,U*d_p] in_dt;  v, z [B,H,d_v] in_dt;  g [B,H] in_dt
+ *   norm_w [d_v] fp32 or NULL;  cape_mask [H] uint8 or NULL
+ *   pos    [B] int32 position of this token in its sequence, or NULL (0)
+ *   S      [B,H,M,d_v] fp32, m [B,H,M] fp32: state, updated in place
+ *   y      [B,H,d_v] out_dt
+ * Errors: INVALID_ARG as above.
+ */
+ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H, ramnet_dtype in_dt,
+                                 const void* k_logits, const void* q_logits, const void* v,
+                                 const void* g, const void* z, const float* norm_w,
+                                 const uint8_t* cape_mask, const int32_t* pos, float* S, float* m,
+                                 void* y, ramnet_dtype out_dt, void* stream);
+
+/*
+ * ramnet_sync_status -- waits for `stream`, then returns RAMNET_ERR_TIMEOUT or
+ * RAMNET_ERR_DEVICE_CHECK if a kernel of this library on the current device recorded a
+ * gave-up wait or a failed check since the last call (and clears the record), or
+ * RAMNET_ERR_CUDA if the stream reports an error; RAMNET_OK otherwise.
+ */
+ramnet_status ramnet_sync_status(void* stream);
+
+/* Message describing the calling thread's last failure ("" if none).  Owned by the
+ * library; valid until the next call from the same thread. */
+const char* ramnet_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RAMNET_H */

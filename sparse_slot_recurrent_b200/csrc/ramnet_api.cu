@@ -1,0 +1,285 @@
+// ramnet_api.cu -- the C ABI declared in include/ramnet.h: argument checks, launches,
+// status reporting.  Nothing here allocates device memory.
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/ramnet.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// Device-side status word of this library (one per device that loads the library).
+__device__ uint32_t g_device_status;
+
+ramnet_status fail(ramnet_status s, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+ramnet_status cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(RAMNET_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(ramnet_dtype d) { return d == RAMNET_F32 || d == RAMNET_BF16; }
+
+// Shared config checks; on success writes M.
+ramnet_status check_config(const ramnet_config* cfg, int* M_out)
+{
+    if (cfg == nullptr) return fail(RAMNET_ERR_INVALID_ARG, "cfg is NULL");
+    if (cfg->d_p < 2 || cfg->d_p > 16) return fail(RAMNET_ERR_INVALID_ARG, "d_p=%d outside [2,16]", cfg->d_p);
+    if (cfg->U < 1 || cfg->U > 8) return fail(RAMNET_ERR_INVALID_ARG, "U=%d outside [1,8]", cfg->U);
+    long long M = 1;
+    for (int u = 0; u < cfg->U; ++u) {
+        M *= cfg->d_p;
+        if (M > 65536) return fail(RAMNET_ERR_INVALID_ARG, "M = d_p^U exceeds 65536");
+    }
+    if (cfg->K < 1 || cfg->K > 64 || cfg->K > M)
+        return fail(RAMNET_ERR_INVALID_ARG, "K=%d outside [1, min(M=%lld, 64)]", cfg->K, M);
+    if (!(cfg->d_v == 16 || cfg->d_v == 32 || cfg->d_v == 64 || cfg->d_v == 128 || cfg->d_v == 256))
+        return fail(RAMNET_ERR_INVALID_ARG, "d_v=%d not in {16,32,64,128,256}", cfg->d_v);
+    if (!(cfg->eps_gsu >= 0.0f) || !(cfg->eps_norm >= 0.0f))
+        return fail(RAMNET_ERR_INVALID_ARG, "epsilons must be >= 0");
+    *M_out = static_cast<int>(M);
+    return RAMNET_OK;
+}
+
+ramnet_status check_sizes(long long B, long long T, long long H)
+{
+    if (B < 1 || T < 1 || H < 1) return fail(RAMNET_ERR_INVALID_ARG, "B, T, H must be >= 1");
+    if (B * T * H > (1ll << 31) - 1) return fail(RAMNET_ERR_INVALID_ARG, "B*T*H too large");
+    return RAMNET_OK;
+}
+
+#define REQUIRE_PTR(p)                                                                          \
+    do {                                                                                        \
+        if ((p) == nullptr) return fail(RAMNET_ERR_INVALID_ARG, "%s is NULL", #p);              \
+        if (!aligned16(p)) return fail(RAMNET_ERR_INVALID_ARG, "%s not 16-byte aligned", #p); \
+    } while (0)
+#define OPTIONAL_PTR(p)                                                                         \
+    do {                                                                                        \
+        if ((p) != nullptr && !aligned16(p))                                                    \
+            return fail(RAMNET_ERR_INVALID_ARG, "%s not 16-byte aligned", #p);                  \
+    } while (0)
+
+uint32_t* device_status_ptr()
+{
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    return static_cast<uint32_t*>(p);
+}
+
+size_t workspace_need(int B, int T, int H, int K)
+{
+    // idx (int32) and weight (fp32) for the key and the query stream
+    const size_t one = static_cast<size_t>(B) * T * H * K * sizeof(int32_t);
+    return 4 * ((one + 255) & ~static_cast<size_t>(255));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ramnet_last_error(void) { return g_last_error.c_str(); }
+
+ramnet_status ramnet_decode_addresses(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, const void* logits,
+                                      ramnet_dtype dt, const int32_t* pos0, const uint8_t* cape_mask,
+                                      int32_t* idx_out, float* w_out, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet_status st = check_config(cfg, &M);
+    if (st != RAMNET_OK) return st;
+    if ((st = check_sizes(B, T, H)) != RAMNET_OK) return st;
+    if (!valid_dtype(dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype %d", static_cast<int>(dt));
+    REQUIRE_PTR(logits);
+    REQUIRE_PTR(idx_out);
+    REQUIRE_PTR(w_out);
+    OPTIONAL_PTR(pos0);
+    OPTIONAL_PTR(cape_mask);
+    ramnet::DecodeParams p{logits, dt == RAMNET_BF16, cfg->d_p, cfg->U, cfg->K, M, cfg->renorm != 0, B, T, H,
+                           pos0, cape_mask, idx_out, w_out};
+    cudaError_t e = ramnet::launch_decode_addresses(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode_addresses launch");
+    return RAMNET_OK;
+}
+
+size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H)
+{
+    int M = 0;
+    if (check_config(cfg, &M) != RAMNET_OK || check_sizes(B, T, H) != RAMNET_OK) return 0;
+    return workspace_need(B, T, H, cfg->K);
+}
+
+ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                                  const void* k_logits, const void* q_logits, const void* v, const void* g,
+                                  const void* z, const float* norm_w, const uint8_t* cape_mask, const int32_t* pos0,
+                                  const float* S_in, const float* m_in, void* y, ramnet_dtype out_dt, float* S_out,
+                                  float* m_out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet_status st = check_config(cfg, &M);
+    if (st != RAMNET_OK) return st;
+    if ((st = check_sizes(B, T, H)) != RAMNET_OK) return st;
+    if (!valid_dtype(in_dt) || !valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
+    REQUIRE_PTR(k_logits);
+    REQUIRE_PTR(q_logits);
+    REQUIRE_PTR(v);
+    REQUIRE_PTR(g);
+    REQUIRE_PTR(z);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(S_out);
+    REQUIRE_PTR(m_out);
+    REQUIRE_PTR(workspace);
+    OPTIONAL_PTR(norm_w);
+    OPTIONAL_PTR(cape_mask);
+    OPTIONAL_PTR(pos0);
+    OPTIONAL_PTR(S_in);
+    OPTIONAL_PTR(m_in);
+    const size_t need = workspace_need(B, T, H, cfg->K);
+    if (workspace_bytes < need)
+        return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+    int ncta = 0, chunk = 0;
+    uint32_t cols = 0;
+    size_t smem = 0;
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, &ncta, &chunk, &cols, &smem))
+        return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", M,
+                    cfg->d_v);
+    uint32_t* status = device_status_ptr();
+    if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+
+    const size_t one = static_cast<size_t>(B) * T * H * cfg->K * sizeof(int32_t);
+    const size_t step = (one + 255) & ~static_cast<size_t>(255);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* widx = reinterpret_cast<int32_t*>(ws);
+    float* wwt = reinterpret_cast<float*>(ws + step);
+    int32_t* ridx = reinterpret_cast<int32_t*>(ws + 2 * step);
+    float* rwt = reinterpret_cast<float*>(ws + 3 * step);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    ramnet::DecodeParams dk{k_logits, in_dt == RAMNET_BF16, cfg->d_p, cfg->U, cfg->K, M, cfg->renorm != 0, B, T, H,
+                            pos0, cape_mask, widx, wwt};
+    cudaError_t e = ramnet::launch_decode_addresses(dk, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: key decode launch");
+    ramnet::DecodeParams dq = dk;
+    dq.logits = q_logits;
+    dq.idx_out = ridx;
+    dq.w_out = rwt;
+    e = ramnet::launch_decode_addresses(dq, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: query decode launch");
+
+    ramnet::ScanParams sp{};
+    sp.widx = widx;
+    sp.wwt = wwt;
+    sp.ridx = ridx;
+    sp.rwt = rwt;
+    sp.v = v;
+    sp.g = g;
+    sp.z = z;
+    sp.in_bf16 = in_dt == RAMNET_BF16;
+    sp.norm_w = norm_w;
+    sp.S_in = S_in;
+    sp.m_in = m_in;
+    sp.y = y;
+    sp.out_bf16 = out_dt == RAMNET_BF16;
+    sp.S_out = S_out;
+    sp.m_out = m_out;
+    sp.B = B;
+    sp.T = T;
+    sp.H = H;
+    sp.K = cfg->K;
+    sp.M = M;
+    sp.d_v = cfg->d_v;
+    sp.ncta = ncta;
+    sp.chunk = chunk;
+    sp.eps_gsu = cfg->eps_gsu;
+    sp.eps_norm = cfg->eps_norm;
+    sp.tmem_cols = cols;
+    sp.status = status;
+    e = ramnet::launch_scan(sp, smem, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return RAMNET_OK;
+}
+
+ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H, ramnet_dtype in_dt,
+                                 const void* k_logits, const void* q_logits, const void* v, const void* g,
+                                 const void* z, const float* norm_w, const uint8_t* cape_mask, const int32_t* pos,
+                                 float* S, float* m, void* y, ramnet_dtype out_dt, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet_status st = check_config(cfg, &M);
+    if (st != RAMNET_OK) return st;
+    if ((st = check_sizes(B, 1, H)) != RAMNET_OK) return st;
+    if (!valid_dtype(in_dt) || !valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
+    REQUIRE_PTR(k_logits);
+    REQUIRE_PTR(q_logits);
+    REQUIRE_PTR(v);
+    REQUIRE_PTR(g);
+    REQUIRE_PTR(z);
+    REQUIRE_PTR(S);
+    REQUIRE_PTR(m);
+    REQUIRE_PTR(y);
+    OPTIONAL_PTR(norm_w);
+    OPTIONAL_PTR(cape_mask);
+    OPTIONAL_PTR(pos);
+    ramnet::StepParams p{};
+    p.k_logits = k_logits;
+    p.q_logits = q_logits;
+    p.v = v;
+    p.g = g;
+    p.z = z;
+    p.in_bf16 = in_dt == RAMNET_BF16;
+    p.norm_w = norm_w;
+    p.cape_mask = cape_mask;
+    p.pos = pos;
+    p.S = S;
+    p.m = m;
+    p.y = y;
+    p.out_bf16 = out_dt == RAMNET_BF16;
+    p.B = B;
+    p.H = H;
+    p.d_p = cfg->d_p;
+    p.U = cfg->U;
+    p.K = cfg->K;
+    p.M = M;
+    p.d_v = cfg->d_v;
+    p.renorm = cfg->renorm != 0;
+    p.eps_gsu = cfg->eps_gsu;
+    p.eps_norm = cfg->eps_norm;
+    cudaError_t e = ramnet::launch_decode_step(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
+    return RAMNET_OK;
+}
+
+ramnet_status ramnet_sync_status(void* stream)
+{
+    g_last_error.clear();
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    uint32_t word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_device_status, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "read status word");
+    if (word != 0) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+        if (word & ramnet::kDevTimeout) return fail(RAMNET_ERR_TIMEOUT, "a device-side wait gave up (status 0x%x)", word);
+        return fail(RAMNET_ERR_DEVICE_CHECK, "a device-side check failed (status 0x%x)", word);
+    }
+    return RAMNET_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+"""The C-ABI library: it loads, exports every symbol include/ramnet.h declares, and its
+host-side argument checks reject bad calls before anything is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from sparse_slot_recurrent_b200 import build as build_mod
+from sparse_slot_recurrent_b200 import ramnet
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ramnet.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return ramnet.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(ramnet_\w+)\s*\(", src, re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    assert set(names) == set(ramnet.EXPORTED), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", build_mod.OUT], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def _cfg(**kw):
+    base = dict(d_p=4, U=5, K=8, d_v=128)
+    base.update(kw)
+    return ramnet.Config(**base)
+
+
+FAKE = 1 << 40  # 16-byte aligned, never dereferenced: every call below fails host-side
+
+
+def _decode(lib, cfg, B=1, T=4, H=1, logits=FAKE, dt=ramnet.RAMNET_BF16, idx=FAKE, w=FAKE, pos0=None):
+    c = cfg._c()
+    return lib.ramnet_decode_addresses(ctypes.byref(c), B, T, H, logits, dt, pos0, None, idx, w, None)
+
+
+@pytest.mark.parametrize("kw", [dict(d_p=1), dict(d_p=17), dict(U=0), dict(U=9), dict(d_p=16, U=5),
+                                dict(K=0), dict(K=65), dict(d_p=2, U=2, K=5), dict(d_v=48), dict(d_v=512),
+                                dict(eps_gsu=-1.0), dict(eps_norm=float("nan"))])
+def test_bad_config_rejected(lib, kw):
+    assert _decode(lib, _cfg(**kw)) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert ramnet.last_error() != ""
+
+
+def test_bad_pointers_and_sizes_rejected(lib):
+    cfg = _cfg()
+    assert _decode(lib, cfg, logits=None) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert "logits" in ramnet.last_error()
+    assert _decode(lib, cfg, logits=FAKE + 4) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert "aligned" in ramnet.last_error()
+    assert _decode(lib, cfg, idx=None) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _decode(lib, cfg, pos0=FAKE + 8) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _decode(lib, cfg, B=0) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _decode(lib, cfg, T=-3) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _decode(lib, cfg, dt=7) == ramnet.RAMNET_ERR_INVALID_ARG
+
+
+def _scan(lib, cfg, B=2, T=8, H=2, ws_bytes=None, S_in=None, y=FAKE, ws=FAKE):
+    c = cfg._c()
+    if ws_bytes is None:
+        ws_bytes = lib.ramnet_scan_workspace_bytes(ctypes.byref(c), B, T, H)
+    return lib.ramnet_scan_forward(ctypes.byref(c), B, T, H, ramnet.RAMNET_BF16, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                   None, None, None, S_in, None, y, ramnet.RAMNET_F32, FAKE, FAKE, ws, ws_bytes,
+                                   None)
+
+
+def test_scan_workspace_size(lib):
+    cfg = _cfg()
+    c = cfg._c()
+    need = lib.ramnet_scan_workspace_bytes(ctypes.byref(c), 8, 4096, 8)
+    assert need >= 4 * 8 * 4096 * 8 * 8 * 4
+    bad = _cfg(d_p=1)._c()
+    assert lib.ramnet_scan_workspace_bytes(ctypes.byref(bad), 8, 4096, 8) == 0
+    assert _scan(lib, cfg, ws_bytes=16) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert "workspace" in ramnet.last_error()
+    assert _scan(lib, cfg, ws=None) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _scan(lib, cfg, y=None) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _scan(lib, cfg, S_in=FAKE + 4) == ramnet.RAMNET_ERR_INVALID_ARG
+
+
+def test_scan_rejects_slot_arrays_beyond_tensor_memory(lib):
+    # M = 65536 slots x 256 channels x 4 B = 64 MiB per head: far beyond 8 SMs of TMEM
+    cfg = _cfg(d_p=16, U=4, K=8, d_v=256)
+    assert _scan(lib, cfg) == ramnet.RAMNET_ERR_UNSUPPORTED
+    assert "tensor memory" in ramnet.last_error()
+
+
+def test_decode_step_checks(lib):
+    cfg = _cfg(d_p=8, U=4, K=16)
+    c = cfg._c()
+    args = [ctypes.byref(c), 4, 2, ramnet.RAMNET_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, FAKE,
+            FAKE, ramnet.RAMNET_F32, None]
+    bad = list(args)
+    bad[12] = None  # S
+    assert lib.ramnet_decode_step(*bad) == ramnet.RAMNET_ERR_INVALID_ARG
+    bad = list(args)
+    bad[1] = 0
+    assert lib.ramnet_decode_step(*bad) == ramnet.RAMNET_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a CUDA device")
+def test_valid_call_without_device_reports_cuda_error(lib):
+    # arguments pass every host check; with no device the first CUDA call fails cleanly
+    assert _decode(lib, _cfg()) == ramnet.RAMNET_ERR_CUDA
+    assert ramnet.last_error() != ""

@@ -1,0 +1,334 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Indices must match bit for bit (including rank order); floating outputs and final state
+within max-abs 1e-5 when every input is fp32 and 1e-3 with bf16 inputs (fp32 state).
+Small cases are compared element by element; the full-size workloads run in the launch
+configuration bench.py times and are compared on sampled tokens / heads, which the
+oracle computes one at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_slot_recurrent_b200 import ramnet
+from sparse_slot_recurrent_b200.workloads import WORKLOADS, Workload, generate, generate_decode_state
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    ramnet.load()
+    yield
+    ramnet.sync_status()
+
+
+def _cfgs(w: Workload, **kw):
+    c = dict(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
+    c.update(kw)
+    return ramnet.Config(**c), oracle.OracleConfig(**c)
+
+
+def _tol(dtype):
+    return TOL_F32 if dtype == torch.float32 else TOL_BF16
+
+
+def _cuda(inp):
+    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items() if not k.startswith("_")}
+
+
+def _maxabs(a, b):
+    a = a.detach().cpu().double().numpy() if torch.is_tensor(a) else a
+    b = b.detach().cpu().double().numpy() if torch.is_tensor(b) else b
+    return float(np.abs(a - b).max()) if a.size else 0.0
+
+
+# ------------------------------------------------------------------ address decoder
+
+DECODE_CASES = [
+    # d_p, U, K, dtype, logit mode
+    (4, 5, 8, torch.float32, "normal"),
+    (4, 5, 8, torch.bfloat16, "ties"),
+    (4, 5, 32, torch.bfloat16, "mixed"),
+    (8, 4, 16, torch.bfloat16, "normal"),
+    (2, 8, 64, torch.float32, "ties"),
+    (16, 4, 64, torch.bfloat16, "normal"),
+    (3, 4, 17, torch.float32, "ties"),
+    (5, 3, 7, torch.bfloat16, "normal"),
+    (16, 2, 1, torch.float32, "normal"),
+    (2, 1, 2, torch.float32, "ties"),
+]
+
+
+def _logits(B, T, H, L, mode, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    if mode == "ties":
+        x = torch.randint(-2, 3, (B, T, H, L), generator=g).float() * 0.25
+    elif mode == "mixed":
+        x = torch.randn((B, T, H, L), generator=g)
+        peaked = torch.rand((B, T, H, 1), generator=g) < 0.7
+        x = x * torch.where(peaked, torch.tensor(4.0), torch.tensor(0.1))
+    else:
+        x = torch.randn((B, T, H, L), generator=g) * 1.5
+    return x.to(dtype).contiguous()
+
+
+@pytest.mark.parametrize("d_p,U,K,dtype,mode", DECODE_CASES)
+def test_decode_addresses_matches_oracle(d_p, U, K, dtype, mode):
+    B, T, H = 2, 37, 3
+    cfg = ramnet.Config(d_p=d_p, U=U, K=K, d_v=16)
+    ocfg = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=16)
+    x = _logits(B, T, H, d_p * U, mode, dtype, seed=d_p * 100 + K)
+    pos0 = torch.tensor([0, 1234567], dtype=torch.int32)
+    mask = torch.tensor([1, 0, 1], dtype=torch.uint8)
+    for renorm in (1, 0):
+        cfg_r = ramnet.Config(d_p=d_p, U=U, K=K, d_v=16, renorm=renorm)
+        ocfg_r = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=16, renorm=renorm)
+        idx, w = ramnet.decode_addresses(cfg_r, x.cuda(), pos0=pos0.cuda(), cape_mask=mask.cuda())
+        oi, ow = oracle.decode_addresses(ocfg_r, x, pos0=pos0, cape_mask=mask)
+        assert np.array_equal(idx.cpu().numpy(), oi)
+        assert _maxabs(w, ow) <= 2e-6
+    del cfg, ocfg
+
+
+@pytest.mark.parametrize("name", ["prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16"])
+def test_decode_addresses_full_size_sampled(name):
+    w = WORKLOADS[name]
+    cfg, ocfg = _cfgs(w)
+    inp = generate(w, seed=0)
+    rng = np.random.default_rng(5)
+    for key in ("k_logits", "q_logits"):
+        x = inp[key]
+        idx, wt = ramnet.decode_addresses(cfg, x.cuda(), pos0=inp["pos0"].cuda(), cape_mask=inp["cape_mask"].cuda())
+        idx, wt = idx.cpu(), wt.cpu()
+        bs = rng.integers(0, w.B, 1500)
+        ts = rng.integers(0, w.T, 1500)
+        hs = rng.integers(0, w.H, 1500)
+        sub = x[bs, ts, hs].reshape(1500, 1, 1, -1)
+        pos = (inp["pos0"][bs].numpy() + ts).astype(np.int32)
+        for n in range(1500):
+            oi, ow = oracle.decode_addresses(ocfg, sub[n:n + 1], pos0=pos[n:n + 1],
+                                             cape_mask=inp["cape_mask"][hs[n]:hs[n] + 1])
+            assert np.array_equal(idx[bs[n], ts[n], hs[n]].numpy(), oi[0, 0, 0]), (key, n)
+            assert _maxabs(wt[bs[n], ts[n], hs[n]], ow[0, 0, 0]) <= 2e-6
+
+
+# ------------------------------------------------------------------ prefill scan
+
+def _oracle_scan(ocfg, inp, norm_w=None, S_in=None, m_in=None):
+    return oracle.scan_forward(ocfg, inp["k_logits"], inp["q_logits"], inp["v"], inp["g"], inp["z"],
+                               norm_w=norm_w, cape_mask=inp["cape_mask"], pos0=inp["pos0"], S_in=S_in, m_in=m_in)
+
+
+def _gpu_scan(cfg, inp, norm_w=None, S_in=None, m_in=None, out_dtype=torch.float32):
+    d = _cuda(inp)
+    y, S, m = ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"],
+                                  norm_w=None if norm_w is None else norm_w.cuda(), cape_mask=d["cape_mask"],
+                                  pos0=d["pos0"], S_in=None if S_in is None else S_in.cuda(),
+                                  m_in=None if m_in is None else m_in.cuda(), out_dtype=out_dtype)
+    ramnet.sync_status()
+    return y.cpu(), S.cpu(), m.cpu()
+
+
+def test_scan_tiny_all_fp32():
+    """The all-fp32 tiny workload, every output element and the final state."""
+    w = WORKLOADS["tiny"]
+    cfg, ocfg = _cfgs(w)
+    inp = generate(w, seed=0)
+    y, S, m = _gpu_scan(cfg, inp)
+    oy, oS, om = _oracle_scan(ocfg, inp)
+    assert _maxabs(y, oy) <= TOL_F32
+    assert _maxabs(S, oS) <= TOL_F32
+    assert _maxabs(m, om) <= TOL_F32
+
+
+SCAN_CASES = [
+    # d_p, U, K, d_v, B, T, H, dtype, cape, with_state, norm_w
+    (4, 5, 8, 128, 2, 211, 3, torch.bfloat16, "mixed", True, True),
+    (4, 5, 32, 128, 1, 150, 2, torch.bfloat16, "off", False, False),
+    (4, 5, 16, 64, 1, 100, 2, torch.float32, "all", True, False),
+    (8, 4, 16, 128, 1, 70, 1, torch.bfloat16, "all", False, False),
+    (4, 4, 8, 32, 2, 90, 2, torch.float32, "mixed", True, True),
+    (2, 8, 64, 16, 1, 80, 1, torch.float32, "off", False, False),
+    (4, 5, 1, 128, 1, 64, 1, torch.float32, "all", True, False),
+    (16, 2, 8, 256, 1, 60, 1, torch.bfloat16, "off", True, True),
+    (3, 5, 7, 32, 1, 77, 2, torch.float32, "mixed", False, False),
+    (4, 5, 8, 128, 1, 1, 1, torch.float32, "all", True, False),
+]
+
+
+def _small_inputs(d_p, U, K, d_v, B, T, H, dtype, cape, seed):
+    w = Workload("case", B=B, H=H, T=T, d_p=d_p, U=U, K=K, d_v=d_v, in_dtype=dtype, cape=cape != "off",
+                 logit_std=1.5)
+    inp = generate(w, seed=seed)
+    if cape == "mixed":
+        inp["cape_mask"] = torch.tensor([(h + 1) % 2 for h in range(H)], dtype=torch.uint8)
+    inp["pos0"] = torch.arange(B, dtype=torch.int32) * 1000 + 3
+    return w, inp
+
+
+@pytest.mark.parametrize("case", SCAN_CASES)
+def test_scan_matches_oracle(case):
+    d_p, U, K, d_v, B, T, H, dtype, cape, with_state, with_nw = case
+    w, inp = _small_inputs(d_p, U, K, d_v, B, T, H, dtype, cape, seed=K + d_v)
+    cfg, ocfg = _cfgs(w)
+    g = torch.Generator().manual_seed(99)
+    S_in = torch.randn((B, H, w.M, d_v), generator=g) if with_state else None
+    m_in = torch.rand((B, H, w.M), generator=g) * 2 if with_state else None
+    nw = torch.rand(d_v, generator=g) + 0.5 if with_nw else None
+    y, S, m = _gpu_scan(cfg, inp, nw, S_in, m_in)
+    oy, oS, om = _oracle_scan(ocfg, inp, nw, S_in, m_in)
+    tol = _tol(dtype)
+    assert _maxabs(y, oy) <= tol
+    assert _maxabs(S, oS) <= tol
+    assert _maxabs(m, om) <= tol
+
+
+def test_scan_unselected_slots_bit_identical():
+    """Rows and masses of slots no token writes come back exactly as they went in."""
+    w, inp = _small_inputs(4, 5, 8, 128, 2, 96, 2, torch.bfloat16, "mixed", seed=3)
+    cfg, _ = _cfgs(w)
+    g = torch.Generator().manual_seed(4)
+    S_in = torch.randn((2, 2, w.M, 128), generator=g)
+    m_in = torch.rand((2, 2, w.M), generator=g)
+    _, S, m = _gpu_scan(cfg, inp, None, S_in, m_in)
+    idx, _ = ramnet.decode_addresses(cfg, inp["k_logits"].cuda(), pos0=inp["pos0"].cuda(),
+                                     cape_mask=inp["cape_mask"].cuda())
+    idx = idx.cpu()
+    for b in range(2):
+        for h in range(2):
+            written = torch.zeros(w.M, dtype=torch.bool)
+            written[idx[b, :, h].reshape(-1).long()] = True
+            assert (~written).sum() > 100
+            assert torch.equal(S[b, h][~written], S_in[b, h][~written])
+            assert torch.equal(m[b, h][~written], m_in[b, h][~written])
+
+
+def test_scan_bf16_output_is_rounded_fp32_output():
+    w, inp = _small_inputs(4, 5, 8, 128, 1, 130, 2, torch.bfloat16, "off", seed=6)
+    cfg, ocfg = _cfgs(w)
+    yb, _, _ = _gpu_scan(cfg, inp, out_dtype=torch.bfloat16)
+    oy, _, _ = _oracle_scan(ocfg, inp)
+    oy = torch.from_numpy(oy)
+    # one bf16 rounding of a value within the bf16-input tolerance
+    assert (yb.double() - oy).abs().max() <= TOL_BF16 + 2.0 ** -8 * oy.abs().max()
+
+
+def test_scan_state_carry_matches_single_call():
+    """scan(T) == scan(T1) then scan(T - T1) with the state and start position carried."""
+    w, inp = _small_inputs(4, 5, 8, 128, 1, 200, 2, torch.float32, "all", seed=7)
+    cfg, _ = _cfgs(w)
+    y, S, m = _gpu_scan(cfg, inp)
+    T1 = 77
+    a = {k: (v[:, :T1] if torch.is_tensor(v) and v.dim() >= 3 else v) for k, v in inp.items()}
+    b = {k: (v[:, T1:].contiguous() if torch.is_tensor(v) and v.dim() >= 3 else v) for k, v in inp.items()}
+    a = {k: (v.contiguous() if torch.is_tensor(v) else v) for k, v in a.items()}
+    b["pos0"] = inp["pos0"] + T1
+    ya, Sa, ma = _gpu_scan(cfg, a)
+    yb, Sb, mb = _gpu_scan(cfg, b, S_in=Sa, m_in=ma)
+    assert _maxabs(torch.cat([ya, yb], 1), y) <= TOL_F32
+    assert _maxabs(Sb, S) <= TOL_F32 and _maxabs(mb, m) <= TOL_F32
+
+
+@pytest.mark.parametrize("name", ["prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16"])
+def test_scan_full_size_sampled_heads(name):
+    """Full workload through the bench's launch configuration; two (b,h) heads compared
+    with the oracle over the whole sequence; every head's never-written rows stay zero."""
+    w = WORKLOADS[name]
+    cfg, ocfg = _cfgs(w)
+    inp = generate(w, seed=0)
+    y, S, m = _gpu_scan(cfg, inp)
+    tol = _tol(w.in_dtype)
+    for (b, h) in [(0, 0), (w.B - 1, w.H - 1)]:
+        sub = {k: inp[k][b:b + 1, :, h:h + 1].contiguous() for k in ("k_logits", "q_logits", "v", "z")}
+        sub["g"] = inp["g"][b:b + 1, :, h:h + 1].contiguous()
+        sub["cape_mask"] = inp["cape_mask"][h:h + 1]
+        sub["pos0"] = inp["pos0"][b:b + 1]
+        oy, oS, om = _oracle_scan(ocfg, sub)
+        assert _maxabs(y[b:b + 1, :, h:h + 1], oy) <= tol
+        assert _maxabs(S[b:b + 1, h:h + 1], oS) <= tol
+        assert _maxabs(m[b:b + 1, h:h + 1], om) <= tol
+    idx, _ = ramnet.decode_addresses(cfg, inp["k_logits"].cuda(), pos0=inp["pos0"].cuda(),
+                                     cape_mask=inp["cape_mask"].cuda())
+    written = torch.zeros((w.B, w.H, w.M), dtype=torch.bool, device="cuda")
+    bi = torch.arange(w.B, device="cuda").view(w.B, 1, 1, 1).expand_as(idx)
+    hi = torch.arange(w.H, device="cuda").view(1, 1, w.H, 1).expand_as(idx)
+    written[bi.reshape(-1), hi.reshape(-1), idx.reshape(-1).long()] = True
+    written = written.cpu()
+    assert (S[~written] == 0).all() and (m[~written] == 0).all()
+
+
+# ------------------------------------------------------------------ decode step
+
+def _decode_inputs(w: Workload, seed):
+    inp = generate(w, seed=seed)
+    S0, m0 = generate_decode_state(w, inp["_gen"])
+    return inp, S0, m0
+
+
+def test_decode_step_matches_oracle_over_steps():
+    w = WORKLOADS["decode_b256"].with_(B=3, H=4, ring=6)
+    cfg, ocfg = _cfgs(w)
+    inp, S0, m0 = _decode_inputs(w, seed=11)
+    mask = torch.tensor([1, 0, 1, 1], dtype=torch.uint8)
+    S, m = S0.cuda(), m0.cuda()
+    oS, om = S0.double().numpy().copy(), m0.double().numpy().copy()
+    for t in range(w.ring):
+        pos = torch.tensor([t, 100 + t, 4095 + t], dtype=torch.int32)
+        step = {k: inp[k][:, t].contiguous() for k in ("k_logits", "q_logits", "v", "g", "z")}
+        y = ramnet.decode_step(cfg, *(step[k].cuda() for k in ("k_logits", "q_logits", "v", "g", "z")), S, m,
+                               pos=pos.cuda(), cape_mask=mask.cuda())
+        oy = oracle.decode_step(ocfg, step["k_logits"], step["q_logits"], step["v"], step["g"], step["z"], oS, om,
+                                pos=pos, cape_mask=mask)
+        ramnet.sync_status()
+        assert _maxabs(y, oy) <= TOL_BF16
+    assert _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
+
+
+def test_decode_step_full_size_sampled_units():
+    """One step of the full batched decode workload (state resident in HBM); sampled
+    (b,h) units are recomputed by the oracle from their pre-step state."""
+    w = WORKLOADS["decode_b256"]
+    cfg, ocfg = _cfgs(w)
+    inp = generate(w, seed=0)
+    gen = torch.Generator(device="cuda").manual_seed(1)
+    S = torch.randn((w.B, w.H, w.M, w.d_v), device="cuda", generator=gen)
+    m = torch.rand((w.B, w.H, w.M), device="cuda", generator=gen) * 1.5 + 0.5
+    units = [(0, 0), (17, 5), (w.B - 1, w.H - 1)]
+    before = {u: (S[u].double().cpu().numpy().copy(), m[u].double().cpu().numpy().copy()) for u in units}
+    pos = torch.arange(w.B, dtype=torch.int32) * 7
+    step = {k: inp[k][:, 3].contiguous() for k in ("k_logits", "q_logits", "v", "g", "z")}
+    y = ramnet.decode_step(cfg, *(step[k].cuda() for k in ("k_logits", "q_logits", "v", "g", "z")), S, m,
+                           pos=pos.cuda(), cape_mask=inp["cape_mask"].cuda())
+    ramnet.sync_status()
+    for (b, h) in units:
+        Sb = before[(b, h)][0][None, None].copy()
+        mb = before[(b, h)][1][None, None].copy()
+        sl = {k: step[k][b:b + 1, h:h + 1] for k in step}
+        oy = oracle.decode_step(ocfg, sl["k_logits"], sl["q_logits"], sl["v"], sl["g"], sl["z"], Sb, mb,
+                                pos=pos[b:b + 1], cape_mask=inp["cape_mask"][h:h + 1])
+        assert _maxabs(y[b, h], oy[0, 0]) <= TOL_BF16
+        assert _maxabs(S[b, h], Sb[0, 0]) <= TOL_BF16
+        assert _maxabs(m[b, h], mb[0, 0]) <= TOL_BF16
+
+
+def test_decode_step_chain_equals_scan():
+    """T single decode steps equal one prefill scan of the same T tokens."""
+    w, inp = _small_inputs(4, 5, 8, 64, 2, 40, 2, torch.float32, "mixed", seed=12)
+    cfg, _ = _cfgs(w)
+    y, S, m = _gpu_scan(cfg, inp)
+    Sd = torch.zeros((2, 2, w.M, 64), device="cuda")
+    md = torch.zeros((2, 2, w.M), device="cuda")
+    d = _cuda(inp)
+    for t in range(40):
+        yd = ramnet.decode_step(cfg, d["k_logits"][:, t].contiguous(), d["q_logits"][:, t].contiguous(),
+                                d["v"][:, t].contiguous(), d["g"][:, t].contiguous(), d["z"][:, t].contiguous(),
+                                Sd, md, pos=d["pos0"] + t, cape_mask=d["cape_mask"])
+        assert _maxabs(yd, y[:, t]) <= TOL_F32
+    assert _maxabs(Sd, S) <= TOL_F32 and _maxabs(md, m) <= TOL_F32
