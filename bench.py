@@ -264,8 +264,9 @@ def run_reference(args, world, rank):
 
 
 def config_of(w, world):
+    io = "bf16" if w.in_dtype == torch.bfloat16 else "fp32"
     return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_p": w.d_p, "U": w.U, "M": w.M, "K": w.K,
-            "d_v": w.d_v, "in_dtype": "bf16", "out_dtype": "bf16", "state": "fp32", "cape": w.cape,
+            "d_v": w.d_v, "in_dtype": io, "out_dtype": io, "state": "fp32", "cape": w.cape,
             "l2": "flushed between timed steps (256 MiB write)",
             "parallelism": f"dp{world} (independent heads per rank, no collective)"}
 
@@ -275,13 +276,14 @@ def config_of(w, world):
 def run_gpu(args, world, rank, local):
     from sparse_slot_recurrent_b200 import ramnet
     ramnet.load()
-    w = WORKLOADS[PREFILL]
+    w = WORKLOADS[args.workload]
     cfg = ramnet.Config(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
     dev = torch.device("cuda", local)
     inp = generate(w, seed=rank)
     host = {k: v.pin_memory() for k, v in inp.items() if torch.is_tensor(v)}
     d = {k: v.to(dev) for k, v in host.items()}
-    y = torch.empty((w.B, w.T, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
+    out_dtype = torch.bfloat16 if w.in_dtype == torch.bfloat16 else torch.float32
+    y = torch.empty((w.B, w.T, w.H, w.d_v), dtype=out_dtype, device=dev)
     S = torch.empty((w.B, w.H, w.M, w.d_v), dtype=torch.float32, device=dev)
     m = torch.empty((w.B, w.H, w.M), dtype=torch.float32, device=dev)
     ws = torch.empty(ramnet.scan_workspace_bytes(cfg, w.B, w.T, w.H), dtype=torch.uint8, device=dev)
@@ -317,7 +319,8 @@ def run_gpu(args, world, rank, local):
 
     # roofline of the timed step against measured HBM bandwidth
     peak, peak_kind = measured_peaks()
-    alg = prefill_algorithmic_bytes(w)
+    nb = 2 if w.in_dtype == torch.bfloat16 else 4
+    alg = prefill_algorithmic_bytes(w, in_bytes=nb, out_bytes=nb)
     achieved = alg / (ms / 1e3) / 1e9
     traffic = recorded_traffic("scan_forward")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
@@ -434,6 +437,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ramnet", "reference"], default="ramnet")
+    ap.add_argument("--workload", default=PREFILL, choices=[k for k, v in WORKLOADS.items() if not v.decode],
+                    help="prefill workload of the timed step (default: the 340M-like Top-8 layer)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
