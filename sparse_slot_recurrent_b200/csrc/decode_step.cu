@@ -15,15 +15,6 @@ namespace {
 
 constexpr int kStepThreads = 128;
 
-__device__ __forceinline__ float step_alpha(float w, float g)
-{
-    g = fminf(fmaxf(g, 0.0f), 1.0f);
-    const float c = g / (1.0f - g);
-    if (w <= 0.0f || c <= 0.0f) return 1.0f;
-    if (w >= 1.0f) return 0.0f;
-    return expf(c * log1pf(-w));
-}
-
 template <int KMAX, int DPMAX>
 __global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
 {
@@ -70,7 +61,7 @@ __global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
         const float g = load_in(p.g, bh, p.in_bf16);
         const int i = wi_s[tid];
         const float w = ww_s[tid];
-        const float mn = step_alpha(w, g) * mrow[i] + w;
+        const float mn = gsu_alpha(w, g) * mrow[i] + w;
         mrow[i] = mn;
         lam_s[tid] = w / (mn + p.eps_gsu);
     }

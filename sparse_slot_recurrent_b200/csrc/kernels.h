@@ -21,13 +21,32 @@ struct DecodeParams {
     float* w_out;              // [B,T,H,K]
 };
 
+// Decode + route (first kernel of the prefill scan): per (b, h, chunk) the token-ordered
+// event list of every owner warp of the scan kernel.
+struct RouteParams {
+    const void* k_logits;  // [B,T,H,U*d_p]
+    const void* q_logits;
+    const void* g;  // [B,T,H]
+    int in_bf16;
+    int d_p, U, K, M, renorm;
+    int B, T, H;
+    const int32_t* pos0;       // [B] or null
+    const uint8_t* cape_mask;  // [H] or null
+    int ncta, cpl, chunk, nchunks;
+    uint2* recs;      // [B*H*nchunks][recs_stride] {meta, weight}
+    float* alphas;    // same indexing: GSU retention of write events
+    long long recs_stride;
+    int* offs;        // [B*H*nchunks][offs_stride]: owner segment starts, then the total
+    long long offs_stride;
+};
+
 struct ScanParams {
-    const int32_t* widx;  // [B,T,H,K] write slots (after CAPE), rank order
-    const float* wwt;     // [B,T,H,K] write weights
-    const int32_t* ridx;  // [B,T,H,K] read slots
-    const float* rwt;     // [B,T,H,K] read weights
+    const uint2* recs;
+    const float* alphas;
+    long long recs_stride;
+    const int* offs;
+    long long offs_stride;
     const void* v;        // [B,T,H,d_v]
-    const void* g;        // [B,T,H]
     const void* z;        // [B,T,H,d_v]
     int in_bf16;
     const float* norm_w;  // [d_v] or null
@@ -43,6 +62,12 @@ struct ScanParams {
     float eps_gsu, eps_norm;
     uint32_t tmem_cols;
     uint32_t* status;
+};
+
+struct ScanPlan {
+    int ncta, chunk, cpl, nchunks;
+    uint32_t tmem_cols;
+    size_t smem_bytes;
 };
 
 struct StepParams {
@@ -64,10 +89,12 @@ struct StepParams {
 };
 
 // Tensor-memory plan of the prefill scan: how many CTAs (cluster size) share one head's
-// slot array and how many TMEM columns each allocates.  Returns false if it does not fit.
-bool scan_plan(int M, int d_v, int K, int* ncta, int* chunk, uint32_t* tmem_cols, size_t* smem_bytes);
+// slot array, the chunk length, and the TMEM columns and shared memory of each CTA.
+// Returns false if the slot array does not fit.
+bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* plan);
 
 cudaError_t launch_decode_addresses(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream);
 cudaError_t launch_decode_step(const StepParams& p, cudaStream_t stream);
 

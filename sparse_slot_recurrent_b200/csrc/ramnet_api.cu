@@ -80,11 +80,28 @@ uint32_t* device_status_ptr()
     return static_cast<uint32_t*>(p);
 }
 
-size_t workspace_need(int B, int T, int H, int K)
+// Scratch of the prefill scan: per (b, h, chunk) the owner-sorted event records, the
+// retention of each write event, and the owner offsets.
+struct WorkspaceLayout {
+    size_t recs, alphas, offs, total;
+    long long recs_stride, offs_stride;
+    int nchunks;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WorkspaceLayout workspace_layout(int B, int T, int H, int K, const ramnet::ScanPlan& plan)
 {
-    // idx (int32) and weight (fp32) for the key and the query stream
-    const size_t one = static_cast<size_t>(B) * T * H * K * sizeof(int32_t);
-    return 4 * ((one + 255) & ~static_cast<size_t>(255));
+    WorkspaceLayout w;
+    w.nchunks = (T + plan.chunk - 1) / plan.chunk;
+    w.recs_stride = static_cast<long long>(round_up(static_cast<size_t>(2 * plan.chunk * K), 4));
+    w.offs_stride = static_cast<long long>(round_up(static_cast<size_t>(8 * plan.ncta + 1), 4));
+    const size_t n = static_cast<size_t>(B) * H * w.nchunks;
+    w.recs = 0;
+    w.alphas = round_up(w.recs + n * w.recs_stride * sizeof(uint2) + 256, 256);
+    w.offs = round_up(w.alphas + n * w.recs_stride * sizeof(float) + 256, 256);
+    w.total = round_up(w.offs + n * w.offs_stride * sizeof(int) + 256, 256);
+    return w;
 }
 
 }  // namespace
@@ -119,7 +136,9 @@ size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t 
 {
     int M = 0;
     if (check_config(cfg, &M) != RAMNET_OK || check_sizes(B, T, H) != RAMNET_OK) return 0;
-    return workspace_need(B, T, H, cfg->K);
+    ramnet::ScanPlan plan;
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, 4, &plan)) return 0;
+    return workspace_layout(B, T, H, cfg->K, plan).total;
 }
 
 ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
@@ -148,45 +167,52 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     OPTIONAL_PTR(pos0);
     OPTIONAL_PTR(S_in);
     OPTIONAL_PTR(m_in);
-    const size_t need = workspace_need(B, T, H, cfg->K);
-    if (workspace_bytes < need)
-        return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
-    int ncta = 0, chunk = 0;
-    uint32_t cols = 0;
-    size_t smem = 0;
-    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, &ncta, &chunk, &cols, &smem))
+    ramnet::ScanPlan plan;
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, 4, &plan))
         return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", M,
                     cfg->d_v);
+    const WorkspaceLayout wl = workspace_layout(B, T, H, cfg->K, plan);
+    if (workspace_bytes < wl.total)
+        return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, wl.total);
     uint32_t* status = device_status_ptr();
     if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-
-    const size_t one = static_cast<size_t>(B) * T * H * cfg->K * sizeof(int32_t);
-    const size_t step = (one + 255) & ~static_cast<size_t>(255);
     char* ws = static_cast<char*>(workspace);
-    int32_t* widx = reinterpret_cast<int32_t*>(ws);
-    float* wwt = reinterpret_cast<float*>(ws + step);
-    int32_t* ridx = reinterpret_cast<int32_t*>(ws + 2 * step);
-    float* rwt = reinterpret_cast<float*>(ws + 3 * step);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    ramnet::DecodeParams dk{k_logits, in_dt == RAMNET_BF16, cfg->d_p, cfg->U, cfg->K, M, cfg->renorm != 0, B, T, H,
-                            pos0, cape_mask, widx, wwt};
-    cudaError_t e = ramnet::launch_decode_addresses(dk, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan: key decode launch");
-    ramnet::DecodeParams dq = dk;
-    dq.logits = q_logits;
-    dq.idx_out = ridx;
-    dq.w_out = rwt;
-    e = ramnet::launch_decode_addresses(dq, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan: query decode launch");
+    ramnet::RouteParams rp{};
+    rp.k_logits = k_logits;
+    rp.q_logits = q_logits;
+    rp.g = g;
+    rp.in_bf16 = in_dt == RAMNET_BF16;
+    rp.d_p = cfg->d_p;
+    rp.U = cfg->U;
+    rp.K = cfg->K;
+    rp.M = M;
+    rp.renorm = cfg->renorm != 0;
+    rp.B = B;
+    rp.T = T;
+    rp.H = H;
+    rp.pos0 = pos0;
+    rp.cape_mask = cape_mask;
+    rp.ncta = plan.ncta;
+    rp.cpl = plan.cpl;
+    rp.chunk = plan.chunk;
+    rp.nchunks = wl.nchunks;
+    rp.recs = reinterpret_cast<uint2*>(ws + wl.recs);
+    rp.alphas = reinterpret_cast<float*>(ws + wl.alphas);
+    rp.recs_stride = wl.recs_stride;
+    rp.offs = reinterpret_cast<int*>(ws + wl.offs);
+    rp.offs_stride = wl.offs_stride;
+    cudaError_t e = ramnet::launch_decode_route(rp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: decode/route launch");
 
     ramnet::ScanParams sp{};
-    sp.widx = widx;
-    sp.wwt = wwt;
-    sp.ridx = ridx;
-    sp.rwt = rwt;
+    sp.recs = rp.recs;
+    sp.alphas = rp.alphas;
+    sp.recs_stride = wl.recs_stride;
+    sp.offs = rp.offs;
+    sp.offs_stride = wl.offs_stride;
     sp.v = v;
-    sp.g = g;
     sp.z = z;
     sp.in_bf16 = in_dt == RAMNET_BF16;
     sp.norm_w = norm_w;
@@ -202,13 +228,13 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     sp.K = cfg->K;
     sp.M = M;
     sp.d_v = cfg->d_v;
-    sp.ncta = ncta;
-    sp.chunk = chunk;
+    sp.ncta = plan.ncta;
+    sp.chunk = plan.chunk;
     sp.eps_gsu = cfg->eps_gsu;
     sp.eps_norm = cfg->eps_norm;
-    sp.tmem_cols = cols;
+    sp.tmem_cols = plan.tmem_cols;
     sp.status = status;
-    e = ramnet::launch_scan(sp, smem, s);
+    e = ramnet::launch_scan(sp, plan.smem_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return RAMNET_OK;
 }

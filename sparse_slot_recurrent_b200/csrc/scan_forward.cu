@@ -2,23 +2,29 @@
 //
 // RAM-Net project page: the three-stage paragraph (decode, CAPE, GSU, then read,
 // normalise, gate), the Gated Sparse Update paragraphs (four steps; unselected slots
-// unchanged) and the GPU-execution paragraph (addresses for all tokens first, then the
-// recurrence over slots whose channels run in parallel).
+// unchanged) and the GPU-execution paragraph (addresses for all tokens first, events
+// grouped by slot, each slot's events in causal order, slots and channels in parallel).
 //
-// Layout.  One head's slot array S [M, d_v] fp32 lives in tensor memory (TMEM) for the
-// whole sequence, spread over a cluster of `ncta` CTAs, one per SM.  Slot i belongs to
-// CTA (i mod ncta) as local slot s = i / ncta; local slot s sits in TMEM lane quadrant
-// (s mod 4), columns [(s/4)*CPL, (s/4)*CPL + CPL), lane l of the quadrant holding
-// channels c*32 + l (c < CPL).  A row access is then one tcgen05.ld/st of CPL columns by
-// the quadrant's warp.  The write mass m of local slots is in shared memory.
-// Warp w serves quadrant w%4 and local slots with ((s/4) mod 2) == w/4, so every slot has
-// exactly one owner warp and the owner applies all events of its slots in token order.
+// State layout.  One head's slot array S [M, d_v] fp32 lives in tensor memory (TMEM) for
+// the whole sequence, spread over a cluster of `ncta` CTAs, one per SM.  Slot i belongs
+// to CTA (i mod ncta) as local slot s = i / ncta, which sits in TMEM lane quadrant
+// (s mod 4), columns [(s/4)*CPL, (s/4)*CPL + CPL); lane l of the quadrant holds channels
+// [l*CPL, l*CPL + CPL).  One slot row is one tcgen05.ld/st of CPL columns by a warp of
+// that quadrant.  Scan warp w (0..7) owns the local slots with s mod 8 == w, and with
+// them their write masses (shared memory).
 //
-// Per chunk of C tokens: stage addresses, gates and values in shared memory; every warp
-// walks the chunk's events in order and applies those it owns (writes: mass, rate,
-// content; reads: weighted row added into the chunk's o buffer); then the CTAs of the
-// cluster exchange partial read sums and squared norms through distributed shared
-// memory and write y for their share of the channels.
+// Work per chunk of C tokens (the decode kernel has already sorted the chunk's events
+// into one token-ordered list per owner warp):
+//   loader warp    bulk-copies this CTA's lists, the write retentions and the chunk's
+//                  value rows into shared memory (2-deep ring);
+//   scan warps     walk their own list in batches of up to 4 events on distinct slots:
+//                  one tcgen05.ld per event, one wait, then writes (mass, rate, content)
+//                  and reads (weighted row red-added into the chunk's o buffer);
+//   epilogue warps add the partial o of all CTAs of the cluster through distributed
+//                  shared memory, exchange the squared norms the same way, and write
+//                  y = o / rms(o) * norm_w * z for this CTA's share of the channels.
+// Every hand-off is an mbarrier; every wait is bounded (about 2 s); a wait that gives up
+// records RAMNET_ERR_TIMEOUT in the status word and the kernel carries on to the end.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,54 +32,52 @@ namespace ramnet {
 
 namespace {
 
-constexpr int kScanThreads = 256;
+constexpr int kScanWarps = 8;
+constexpr int kLoadWarp = 8;
+constexpr int kEpiWarp0 = 9;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = (kScanWarps + 1 + kEpiWarps) * 32;
+
+enum Bar { kStage = 0, kScan = 2, kOFree = 4, kZ = 6, kPeerO = 8, kPeerSS = 10, kFin = 12, kNumBars = 13 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
-struct ScanLayout {
-    size_t bar, holder, ok, m, widx, wwt, ridx, rwt, g, ss, vbuf, obuf, total;
+struct Layout {
+    size_t bars, holder, m, offs, recs, alph, vbuf, zbuf, obuf, ss, total;
+    size_t recs_bytes, alph_bytes, vbuf_bytes, zbuf_bytes, obuf_bytes;
 };
 
-__host__ __device__ inline ScanLayout scan_layout(int Ml, int C, int K, int dv)
+__host__ __device__ inline Layout scan_layout(int Ml, int C, int K, int dv, int ncta, int es)
 {
-    ScanLayout L;
+    Layout L;
+    L.recs_bytes = align16(sizeof(uint2) * (2 * C * K + 4));
+    L.alph_bytes = align16(sizeof(float) * (2 * C * K + 8));
+    L.vbuf_bytes = align16(static_cast<size_t>(C) * dv * es);
+    L.zbuf_bytes = align16(static_cast<size_t>(C) * (dv / ncta) * es);
+    L.obuf_bytes = align16(sizeof(float) * C * dv);
     size_t o = 0;
-    L.bar = o;
-    o += 8;
+    L.bars = o;
+    o += align16(8 * kNumBars);
     L.holder = o;
-    o += 4;
-    L.ok = o;
-    o += 4;
+    o += 16;
+    L.offs = o;  // per buffer: 9 owner offsets + record base + alpha base
+    o += align16(sizeof(int) * 2 * 12);
     L.m = o;
     o += align16(sizeof(float) * Ml);
-    L.widx = o;
-    o += align16(sizeof(int32_t) * C * K);
-    L.wwt = o;
-    o += align16(sizeof(float) * C * K);
-    L.ridx = o;
-    o += align16(sizeof(int32_t) * C * K);
-    L.rwt = o;
-    o += align16(sizeof(float) * C * K);
-    L.g = o;
-    o += align16(sizeof(float) * C);
+    L.recs = o;
+    o += 2 * L.recs_bytes;
+    L.alph = o;
+    o += 2 * L.alph_bytes;
+    L.vbuf = o;
+    o += 2 * L.vbuf_bytes;
+    L.zbuf = o;
+    o += 2 * L.zbuf_bytes;
+    L.obuf = o;
+    o += 2 * L.obuf_bytes;
     L.ss = o;
     o += align16(sizeof(float) * 2 * C);
-    L.vbuf = o;
-    o += align16(sizeof(float) * C * dv);
-    L.obuf = o;
-    o += align16(sizeof(float) * C * dv);
     L.total = o;
     return L;
-}
-
-// Gated Sparse Update, step 1 (retention): (1 - w)^(g/(1-g)), g clamped to [0,1].
-__device__ __forceinline__ float gsu_alpha(float w, float g)
-{
-    g = fminf(fmaxf(g, 0.0f), 1.0f);
-    const float c = g / (1.0f - g);
-    if (w <= 0.0f || c <= 0.0f) return 1.0f;
-    if (w >= 1.0f) return 0.0f;
-    return expf(c * log1pf(-w));
 }
 
 __device__ __forceinline__ uint64_t global_ns()
@@ -83,230 +87,390 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// Cluster-wide rendezvous on this CTA's mbarrier with a bounded wait (about 2 s).
-// Thread 0 arrives on every CTA's barrier and waits; the verdict is broadcast to the CTA.
-__device__ bool cluster_point(uint64_t* bar, uint32_t& phase, int ncta, int* ok_s, uint32_t* status)
+__device__ __forceinline__ bool try_wait_cta(uint32_t bar, uint32_t parity)
 {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int ok = *ok_s;
-        if (ok) {
-            const uint32_t a = smem_addr(bar);
-            for (int r = 0; r < ncta; ++r) mbar_arrive_cluster(map_to_rank(a, static_cast<uint32_t>(r)));
-            ok = 0;
-            const uint64_t t_end = global_ns() + 2000000000ull;
-            for (uint32_t it = 0; it < kSpinLimit; ++it) {
-                if (mbar_try_wait_cluster(bar, phase & 1u)) {
-                    ok = 1;
-                    break;
-                }
-                if ((it & 255u) == 255u && global_ns() > t_end) break;
-            }
-            if (!ok) set_status(status, kDevTimeout);
-        }
-        *ok_s = ok;
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool try_wait_clu(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase `parity` of the mbarrier at shared address `bar`: at most
+// kSpinLimit polls and about 2 s.  On expiry the status word gets kDevTimeout and the
+// CTA's abort flag is raised, after which every later wait of the CTA returns at once,
+// so a kernel that lost a signal still ends within a few seconds.
+template <bool kCluster>
+__device__ __noinline__ void wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag)
+{
+    if (*abort_flag) return;
+    const uint64_t t_end = global_ns() + 2000000000ull;
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        if (kCluster ? try_wait_clu(bar, parity) : try_wait_cta(bar, parity)) return;
+        if ((it & 1023u) == 1023u && (global_ns() > t_end || *abort_flag)) break;
     }
-    ++phase;
-    __syncthreads();
-    return *ok_s != 0;
+    *abort_flag = 1;
+    set_status(status, kDevTimeout);
+}
+
+// Before exit: wait (bounded, ignoring the abort flag) until the bulk copies this CTA
+// issued into its own shared memory have landed.
+__device__ __noinline__ void drain_copies(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t_end = global_ns() + 2000000000ull;
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        if (try_wait_cta(bar, parity)) return;
+        if ((it & 1023u) == 1023u && global_ns() > t_end) return;
+    }
+}
+
+__device__ __forceinline__ void arrive_cta(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on mbarrier `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
+
+// Cluster-wide signal: one thread arrives on the same mbarrier of every CTA.
+__device__ __forceinline__ void signal_cluster(uint32_t bar, int ncta)
+{
+    for (int r = 0; r < ncta; ++r) mbar_arrive_cluster(map_to_rank(bar, static_cast<uint32_t>(r)));
+}
+
+// CPL consecutive input elements (fp32 or bf16) from shared memory, as fp32.
+template <int CPL>
+__device__ __forceinline__ void load_row(const unsigned char* base, int elem, int is_bf16, float (&v)[CPL])
+{
+    if (is_bf16) {
+        const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(base) + elem;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) v[c] = __bfloat162float(pb[c]);
+    } else {
+        const float* pf = reinterpret_cast<const float*>(base) + elem;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) v[c] = pf[c];
+    }
 }
 
 template <int CPL>
-__global__ void __launch_bounds__(kScanThreads, 1) k_scan_tmem(ScanParams p)
+__global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int C = p.chunk, K = p.K, dv = p.d_v, ncta = p.ncta, M = p.M;
-    const int LW = dv < 32 ? dv : 32;  // active lanes per row
+    const int C = p.chunk, dv = p.d_v, ncta = p.ncta, M = p.M;
+    const int LW = dv < 32 ? dv : 32;  // lanes holding channels
+    const int es = p.in_bf16 ? 2 : 4;
+    const int Dr = dv / ncta;          // output channels of this CTA
     const uint32_t rank = ncta > 1 ? cluster_ctarank() : 0u;
     const int bh = blockIdx.x / ncta;
-    const int b = bh / p.H, h = bh % p.H;
+    const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int q = warp & 3, sub = warp >> 2;
     const int Ml = (M - static_cast<int>(rank) + ncta - 1) / ncta;
-    const ScanLayout L = scan_layout((M + ncta - 1) / ncta, C, K, dv);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
+    const int nch = (p.T + C - 1) / C;
+    const Layout L = scan_layout((M + ncta - 1) / ncta, C, p.K, dv, ncta, es);
+    const uint32_t bars = smem_addr(smem + L.bars);
+    auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
     uint32_t* holder = reinterpret_cast<uint32_t*>(smem + L.holder);
-    int* ok_s = reinterpret_cast<int*>(smem + L.ok);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.holder + 4);
+    int* offs_s = reinterpret_cast<int*>(smem + L.offs);
     float* m_s = reinterpret_cast<float*>(smem + L.m);
-    int32_t* widx_s = reinterpret_cast<int32_t*>(smem + L.widx);
-    float* wwt_s = reinterpret_cast<float*>(smem + L.wwt);
-    int32_t* ridx_s = reinterpret_cast<int32_t*>(smem + L.ridx);
-    float* rwt_s = reinterpret_cast<float*>(smem + L.rwt);
-    float* g_s = reinterpret_cast<float*>(smem + L.g);
     float* ss_s = reinterpret_cast<float*>(smem + L.ss);
-    float* vbuf = reinterpret_cast<float*>(smem + L.vbuf);
-    float* obuf = reinterpret_cast<float*>(smem + L.obuf);
 
     if (tid == 0) {
-        *ok_s = 1;
-        if (ncta > 1) {
-            mbar_init(bar, static_cast<uint32_t>(ncta));
-            fence_mbar_init_cluster();
+        *abort_flag = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kStage + i, 1);
+            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kScan + i, kScanWarps * 32);
+            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kOFree + i, kEpiWarps * 32);
+            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kZ + i, 1);
+            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kPeerO + i, static_cast<uint32_t>(ncta));
+            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kPeerSS + i, static_cast<uint32_t>(ncta));
         }
+        mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kFin, static_cast<uint32_t>(ncta));
+        fence_mbar_init_cluster();
     }
     if (warp == 0) tmem_alloc(holder, p.tmem_cols);
+    // zero both o buffers and the masses / initial state
+    {
+        float4* ob = reinterpret_cast<float4*>(smem + L.obuf);
+        for (size_t i = tid; i < 2 * L.obuf_bytes / 16; i += kThreads) ob[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = tid; s < Ml; s += kThreads)
+            m_s[s] = p.m_in != nullptr ? p.m_in[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] : 0.0f;
+    }
     tmem_fence_before_sync();
     __syncthreads();
     if (ncta > 1) cluster_sync_all();
     tmem_fence_after_sync();
     const uint32_t tbase = *holder;
-    const uint32_t tq = static_cast<uint32_t>(32 * q) << 16;
 
-    // ---- initial state: owned rows into TMEM, masses into shared memory
-    for (int s = 4 * sub + q; s < Ml; s += 8) {
-        const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
-        float r[CPL];
+    if (warp < kScanWarps) {
+        // ============================================================ scan warps
+        const int q = warp & 3;
+        const uint32_t tq = tbase + (static_cast<uint32_t>(32 * q) << 16);
+        for (int s = warp; s < Ml; s += 8) {
+            const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
+            float r[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) r[c] = (p.S_in != nullptr && lane < LW) ? p.S_in[row + c * LW + lane] : 0.0f;
-        tmem_st<CPL>(tbase + tq + static_cast<uint32_t>((s >> 2) * CPL), r);
-    }
-    tmem_wait_st();
-    for (int s = tid; s < Ml; s += kScanThreads)
-        m_s[s] = p.m_in != nullptr ? p.m_in[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] : 0.0f;
-    __syncthreads();
-
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int t0 = 0; t0 < p.T && ok; t0 += C) {
-        const int n = min(C, p.T - t0);
-        float* ss = ss_s + ((t0 / C) & 1) * C;
-        // ---- stage the chunk
-        for (int e = tid; e < n * K; e += kScanThreads) {
-            const int t = e / K, j = e - (e / K) * K;
-            const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
-            widx_s[e] = p.widx[th * K + j];
-            wwt_s[e] = p.wwt[th * K + j];
-            ridx_s[e] = p.ridx[th * K + j];
-            rwt_s[e] = p.rwt[th * K + j];
+            for (int c = 0; c < CPL; ++c) r[c] = (p.S_in != nullptr && lane < LW) ? p.S_in[row + lane * CPL + c] : 0.0f;
+            tmem_st<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), r);
         }
-        for (int t = tid; t < n; t += kScanThreads) {
-            const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
-            g_s[t] = load_in(p.g, th, p.in_bf16);
-            ss[t] = 0.0f;
-        }
-        for (int e = tid; e < n * dv; e += kScanThreads) {
-            const int t = e / dv, ch = e - (e / dv) * dv;
-            const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
-            vbuf[t * dv + (ch % LW) * CPL + ch / LW] = load_in(p.v, th * dv + ch, p.in_bf16);
-            obuf[e] = 0.0f;
-        }
-        __syncthreads();
-
-        // ---- events of the chunk, in token order; writes of a token before its reads
-        for (int t = 0; t < n; ++t) {
-            const float g = g_s[t];
-            for (int grp = 0; grp < 2 * K; grp += 32) {
-                const int e = grp + lane;
-                const bool valid = e < 2 * K;
-                const bool is_w = e < K;
-                const int j = is_w ? e : e - K;
-                int slot = 0;
-                float coef = 0.0f;
-                if (valid) {
-                    slot = is_w ? widx_s[t * K + j] : ridx_s[t * K + j];
-                    coef = is_w ? wwt_s[t * K + j] : rwt_s[t * K + j];
-                }
-                const int s_loc = slot / ncta;
-                const bool own = valid && (slot - s_loc * ncta) == static_cast<int>(rank) && (s_loc & 3) == q &&
-                                 ((s_loc >> 2) & 1) == sub;
-                uint32_t mask = __ballot_sync(0xffffffffu, own);
-                while (mask) {
-                    const int src = __ffs(mask) - 1;
-                    mask &= mask - 1;
-                    const int sl = __shfl_sync(0xffffffffu, s_loc, src);
-                    const float cf = __shfl_sync(0xffffffffu, coef, src);
-                    const uint32_t taddr = tbase + tq + static_cast<uint32_t>((sl >> 2) * CPL);
-                    float S[CPL];
-                    tmem_ld<CPL>(taddr, S);
-                    tmem_wait_ld();
-                    if (grp + src < K) {
-                        // Gated Sparse Update steps 1-4 for this slot
-                        const float mo = m_s[sl];
-                        const float a = gsu_alpha(cf, g);
-                        const float mn = a * mo + cf;
-                        const float lam = cf / (mn + p.eps_gsu);
-                        __syncwarp();
-                        if (lane == 0) m_s[sl] = mn;
-                        __syncwarp();
-#pragma unroll
-                        for (int c = 0; c < CPL; ++c) {
-                            const float vv = lane < LW ? vbuf[t * dv + lane * CPL + c] : 0.0f;
-                            S[c] = fmaf(lam, vv - S[c], S[c]);
+        tmem_wait_st();
+        for (int c = 0; c < nch; ++c) {
+            const int bf = c & 1;
+            wait_bounded<false>(bar(kStage + bf), (c >> 1) & 1, p.status, abort_flag);
+            if (c >= 2) wait_bounded<false>(bar(kOFree + bf), ((c - 2) >> 1) & 1, p.status, abort_flag);
+            const uint2* recs = reinterpret_cast<const uint2*>(smem + L.recs + bf * L.recs_bytes);
+            const float* alph = reinterpret_cast<const float*>(smem + L.alph + bf * L.alph_bytes);
+            const unsigned char* vb = smem + L.vbuf + bf * L.vbuf_bytes;
+            float* ob = reinterpret_cast<float*>(smem + L.obuf + bf * L.obuf_bytes);
+            const int* ofs = offs_s + bf * 12;
+            const int rbase = ofs[9], abase = ofs[10];
+            const int end = ofs[warp + 1] - rbase;
+            const int ashift = rbase - abase;
+            for (int i = ofs[warp] - rbase; i < end;) {
+                // a batch of up to 4 events on distinct slots (columns)
+                uint2 r[4];
+                r[0] = recs[i];
+                int nb = 1;
+                if (i + 1 < end) {
+                    r[1] = recs[i + 1];
+                    const uint32_t c0 = r[0].x & 0x7FFFu, c1 = r[1].x & 0x7FFFu;
+                    if (c1 != c0) {
+                        nb = 2;
+                        if (i + 2 < end) {
+                            r[2] = recs[i + 2];
+                            const uint32_t c2 = r[2].x & 0x7FFFu;
+                            if (c2 != c0 && c2 != c1) {
+                                nb = 3;
+                                if (i + 3 < end) {
+                                    r[3] = recs[i + 3];
+                                    const uint32_t c3 = r[3].x & 0x7FFFu;
+                                    if (c3 != c0 && c3 != c1 && c3 != c2) nb = 4;
+                                }
+                            }
                         }
-                        tmem_st<CPL>(taddr, S);
-                        tmem_wait_st();
-                    } else if (lane < LW) {
-#pragma unroll
-                        for (int c = 0; c < CPL; ++c) atomicAdd(&obuf[t * dv + lane * CPL + c], cf * S[c]);
                     }
                 }
+                float S[4][CPL];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < nb) tmem_ld<CPL>(tq + (r[k].x & 0x7FFFu), S[k]);
+                // masses and rates of the batch's writes while the loads are in flight
+                float lam[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    lam[k] = 0.0f;
+                    if (k < nb && (r[k].x & 0x8000u)) {
+                        const int s = 4 * static_cast<int>((r[k].x & 0x7FFFu) / CPL) + q;
+                        const float w = __uint_as_float(r[k].y);
+                        const float mn = alph[i + k + ashift] * m_s[s] + w;
+                        lam[k] = w * __frcp_rn(mn + p.eps_gsu);
+                        __syncwarp();
+                        if (lane == 0) m_s[s] = mn;
+                    }
+                }
+                __syncwarp();
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    if (k < nb) {
+                        const int t = static_cast<int>(r[k].x >> 16);
+                        if (r[k].x & 0x8000u) {
+                            float vv[CPL];
+                            load_row<CPL>(vb, t * dv + (lane < LW ? lane : 0) * CPL, p.in_bf16, vv);
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) S[k][cc] = fmaf(lam[k], vv[cc] - S[k][cc], S[k][cc]);
+                            tmem_st<CPL>(tq + (r[k].x & 0x7FFFu), S[k]);
+                        } else if (lane < LW) {
+                            const float rw = __uint_as_float(r[k].y);
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) atomicAdd(&ob[t * dv + cc * LW + lane], rw * S[k][cc]);
+                        }
+                    }
+                }
+                tmem_wait_st();
+                i += nb;
+            }
+            arrive_cta(bar(kScan + bf));
+        }
+        // final state of the owned slots
+        for (int s = warp; s < Ml; s += 8) {
+            const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
+            float r[CPL];
+            tmem_ld<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), r);
+            tmem_wait_ld();
+            if (lane < LW) {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) p.S_out[row + lane * CPL + c] = r[c];
+            }
+            if (lane == 0) p.m_out[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] = m_s[s];
+        }
+    } else if (warp == kLoadWarp) {
+        // ============================================================ loader warp
+        for (int c = 0; c < nch; ++c) {
+            const int bf = c & 1;
+            const int n = min(C, p.T - c * C);
+            if (c >= 2) {
+                wait_bounded<false>(bar(kScan + bf), ((c - 2) >> 1) & 1, p.status, abort_flag);
+                fence_proxy_async();
+            }
+            const long long chunk = static_cast<long long>(bh) * nch + c;
+            const int* og = p.offs + chunk * p.offs_stride + 8 * rank;
+            const int o = lane < 9 ? og[lane] : 0;
+            const int lo = __shfl_sync(0xffffffffu, o, 0), hi = __shfl_sync(0xffffffffu, o, 8);
+            const int lo_r = lo & ~1, lo_a = lo & ~3;
+            const uint32_t rb = hi > lo ? static_cast<uint32_t>(align16(static_cast<size_t>(hi - lo_r) * 8)) : 0u;
+            const uint32_t ab = hi > lo ? static_cast<uint32_t>(align16(static_cast<size_t>(hi - lo_a) * 4)) : 0u;
+            const uint32_t vrow = static_cast<uint32_t>(dv * es);
+            int* ofs = offs_s + bf * 12;
+            if (lane < 9) ofs[lane] = o;
+            if (lane == 9) ofs[9] = lo_r;
+            if (lane == 10) ofs[10] = lo_a;
+            __syncwarp();
+            if (lane == 0) arrive_expect_tx(bar(kStage + bf), rb + ab + static_cast<uint32_t>(n) * vrow);
+            __syncwarp();
+            if (lane == 0 && rb) bulk_g2s(smem_addr(smem + L.recs + bf * L.recs_bytes), p.recs + chunk * p.recs_stride + lo_r, rb, bar(kStage + bf));
+            if (lane == 1 && ab) bulk_g2s(smem_addr(smem + L.alph + bf * L.alph_bytes), p.alphas + chunk * p.recs_stride + lo_a, ab, bar(kStage + bf));
+            for (int t = lane; t < n; t += 32) {
+                const size_t th = (static_cast<size_t>(b) * p.T + c * C + t) * p.H + h;
+                bulk_g2s(smem_addr(smem + L.vbuf + bf * L.vbuf_bytes + static_cast<size_t>(t) * vrow),
+                         static_cast<const unsigned char*>(p.v) + th * vrow, vrow, bar(kStage + bf));
             }
         }
-        __syncthreads();
-
-        // ---- read sums across the cluster, RMSNorm, gate, y
-        if (ncta == 1) {
-            for (int e = tid; e < n * dv; e += kScanThreads) {
-                const int t = e / dv, ch = e - (e / dv) * dv;
-                const float o = obuf[t * dv + (ch % LW) * CPL + ch / LW];
-                atomicAdd(&ss[t], o * o);
+    } else {
+        // ============================================================ epilogue warps
+        const int e = warp - kEpiWarp0;
+        const int etid = tid - kEpiWarp0 * 32;
+        const int cpl_lane = Dr >= 32 ? Dr / 32 : 1;  // output channels per lane
+        const bool lane_on = lane * cpl_lane < Dr;
+        const int ch0 = static_cast<int>(rank) * Dr + lane * cpl_lane;
+        const uint32_t zrow = static_cast<uint32_t>(Dr * es);
+        for (int c = 0; c < nch; ++c) {
+            const int bf = c & 1;
+            const int n = min(C, p.T - c * C);
+            const int t0 = c * C;
+            // stage z (this CTA's channels) for the chunk
+            if (e == 0) {
+                fence_proxy_async();
+                if (lane == 0) arrive_expect_tx(bar(kZ + bf), static_cast<uint32_t>(n) * zrow);
+                __syncwarp();
+                for (int t = lane; t < n; t += 32) {
+                    const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
+                    bulk_g2s(smem_addr(smem + L.zbuf + bf * L.zbuf_bytes + static_cast<size_t>(t) * zrow),
+                             static_cast<const unsigned char*>(p.z) + (th * dv + static_cast<size_t>(rank) * Dr) * es,
+                             zrow, bar(kZ + bf));
+                }
             }
-            __syncthreads();
-        } else {
-            ok = cluster_point(bar, phase, ncta, ok_s, p.status);
-            if (!ok) break;
-            const int Dr = dv / ncta;
-            for (int e = tid; e < n * Dr; e += kScanThreads) {
-                const int t = e / Dr, ch = static_cast<int>(rank) * Dr + (e - (e / Dr) * Dr);
-                const int pos = t * dv + (ch % LW) * CPL + ch / LW;
-                const uint32_t a = smem_addr(&obuf[pos]);
-                float o = 0.0f;
-                for (int r = 0; r < ncta; ++r) o += ld_cluster_f32(map_to_rank(a, static_cast<uint32_t>(r)));
-                obuf[pos] = o;
-                atomicAdd(&ss[t], o * o);
+            wait_bounded<false>(bar(kScan + bf), (c >> 1) & 1, p.status, abort_flag);
+            float* ob = reinterpret_cast<float*>(smem + L.obuf + bf * L.obuf_bytes);
+            float* ss = ss_s + bf * C;
+            // all CTAs' partial sums of this chunk are complete
+            if (etid == 0) {
+                if (ncta == 1) arrive_cta(bar(kPeerO + bf));
+                else signal_cluster(bar(kPeerO + bf), ncta);
             }
-            ok = cluster_point(bar, phase, ncta, ok_s, p.status);
-            if (!ok) break;
-        }
-        {
-            const int Dr = dv / ncta;
-            for (int e = tid; e < n * Dr; e += kScanThreads) {
-                const int t = e / Dr, ch = static_cast<int>(rank) * Dr + (e - (e / Dr) * Dr);
-                const int pos = t * dv + (ch % LW) * CPL + ch / LW;
-                float tot;
+            wait_bounded<true>(bar(kPeerO + bf), (c >> 1) & 1, p.status, abort_flag);
+            for (int t = e; t < n; t += kEpiWarps) {
+                float sq = 0.0f;
+                if (lane_on) {
+                    for (int k = 0; k < cpl_lane; ++k) {
+                        const int ch = ch0 + k;
+                        const int pos = t * dv + (ch % CPL) * LW + ch / CPL;
+                        float o = 0.0f;
+                        if (ncta == 1) {
+                            o = ob[pos];
+                        } else {
+                            const uint32_t a = smem_addr(&ob[pos]);
+                            for (int r = 0; r < ncta; ++r) o += ld_cluster_f32(map_to_rank(a, static_cast<uint32_t>(r)));
+                            ob[pos] = o;
+                        }
+                        sq += o * o;
+                    }
+                }
+#pragma unroll
+                for (int d = 16; d > 0; d >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, d);
+                if (lane == 0) ss[t] = sq;
+            }
+            epi_barrier();
+            if (etid == 0) {
+                if (ncta == 1) arrive_cta(bar(kPeerSS + bf));
+                else signal_cluster(bar(kPeerSS + bf), ncta);
+            }
+            wait_bounded<true>(bar(kPeerSS + bf), (c >> 1) & 1, p.status, abort_flag);
+            wait_bounded<false>(bar(kZ + bf), (c >> 1) & 1, p.status, abort_flag);
+            const unsigned char* zb = smem + L.zbuf + bf * L.zbuf_bytes;
+            for (int t = e; t < n; t += kEpiWarps) {
+                float tot = 0.0f;
                 if (ncta == 1) {
                     tot = ss[t];
                 } else {
-                    tot = 0.0f;
                     const uint32_t a = smem_addr(&ss[t]);
                     for (int r = 0; r < ncta; ++r) tot += ld_cluster_f32(map_to_rank(a, static_cast<uint32_t>(r)));
                 }
                 const float inv = 1.0f / sqrtf(tot / dv + p.eps_norm);
-                const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
-                const float nw = p.norm_w != nullptr ? p.norm_w[ch] : 1.0f;
-                const float y = obuf[pos] * inv * nw * load_in(p.z, th * dv + ch, p.in_bf16);
-                store_out(p.y, th * dv + ch, y, p.out_bf16);
+                if (lane_on) {
+                    const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
+                    for (int k = 0; k < cpl_lane; ++k) {
+                        const int ch = ch0 + k;
+                        const int pos = t * dv + (ch % CPL) * LW + ch / CPL;
+                        const float zz = p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(zb)[t * Dr + ch - static_cast<int>(rank) * Dr])
+                                                   : reinterpret_cast<const float*>(zb)[t * Dr + ch - static_cast<int>(rank) * Dr];
+                        const float nw = p.norm_w != nullptr ? p.norm_w[ch] : 1.0f;
+                        store_out(p.y, th * dv + ch, ob[pos] * inv * nw * zz, p.out_bf16);
+                    }
+                }
             }
-        }
-        __syncthreads();
-    }
-
-    // ---- final state out
-    for (int s = 4 * sub + q; s < Ml; s += 8) {
-        const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
-        float r[CPL];
-        tmem_ld<CPL>(tbase + tq + static_cast<uint32_t>((s >> 2) * CPL), r);
-        tmem_wait_ld();
-        if (lane < LW) {
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) p.S_out[row + c * LW + lane] = r[c];
+            // every CTA has read this chunk's partial sums and every epilogue warp has
+            // written its y: clear them for chunk c + 2
+            epi_barrier();
+            float4* ob4 = reinterpret_cast<float4*>(ob);
+            for (size_t i = etid; i < L.obuf_bytes / 16; i += kEpiWarps * 32) ob4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            arrive_cta(bar(kOFree + bf));
         }
     }
-    for (int s = tid; s < Ml; s += kScanThreads)
-        p.m_out[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] = m_s[s];
 
+    // copies still in flight after an abort must land before the CTA exits
+    if (warp == kLoadWarp || warp == kEpiWarp0) {
+        const int base = warp == kLoadWarp ? kStage : kZ;
+        for (int c = max(0, nch - 2); c < nch; ++c) drain_copies(bar(base + (c & 1)), (c >> 1) & 1);
+    }
     // no CTA leaves while a peer may still read its shared memory
-    if (ncta > 1 && ok) cluster_point(bar, phase, ncta, ok_s, p.status);
+    __syncthreads();
+    if (ncta > 1 && tid == 0) {
+        signal_cluster(bar(kFin), ncta);
+        wait_bounded<true>(bar(kFin), 0, p.status, abort_flag);
+    }
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
@@ -315,7 +479,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_tmem(ScanParams p)
 
 }  // namespace
 
-bool scan_plan(int M, int d_v, int K, int* ncta, int* chunk, uint32_t* tmem_cols, size_t* smem_bytes)
+bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
 {
     const int cpl = d_v < 32 ? 1 : d_v / 32;
     int n = 0;
@@ -333,14 +497,16 @@ bool scan_plan(int M, int d_v, int K, int* ncta, int* chunk, uint32_t* tmem_cols
     uint32_t alloc = 32;
     while (alloc < static_cast<uint32_t>(cols)) alloc <<= 1;
     int C = 64;
-    while (C > 8 && scan_layout(Ml, C, K, d_v).total > 200 * 1024) C >>= 1;
-    const size_t total = scan_layout(Ml, C, K, d_v).total;
+    while (C > 8 && (2 * C * K > 2048 || scan_layout(Ml, C, K, d_v, n, in_bytes).total > 200 * 1024)) C >>= 1;
+    const size_t total = scan_layout(Ml, C, K, d_v, n, in_bytes).total;
     if (total > 200 * 1024) return false;
-    *ncta = n;
-    *chunk = C;
-    *tmem_cols = alloc;
+    out->ncta = n;
+    out->chunk = C;
+    out->cpl = cpl;
+    out->tmem_cols = alloc;
     // more than half of the SM's shared memory: exactly one CTA (and one TMEM owner) per SM
-    *smem_bytes = total < 116 * 1024 ? 116 * 1024 : total;
+    out->smem_bytes = total < 116 * 1024 ? 116 * 1024 : total;
+    out->nchunks = 0;
     return true;
 }
 
@@ -348,17 +514,17 @@ cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t str
 {
     void (*kern)(ScanParams) = nullptr;
     switch (p.d_v < 32 ? 1 : p.d_v / 32) {
-        case 1: kern = k_scan_tmem<1>; break;
-        case 2: kern = k_scan_tmem<2>; break;
-        case 4: kern = k_scan_tmem<4>; break;
-        case 8: kern = k_scan_tmem<8>; break;
+        case 1: kern = k_scan<1>; break;
+        case 2: kern = k_scan<2>; break;
+        case 4: kern = k_scan<4>; break;
+        case 8: kern = k_scan<8>; break;
         default: return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.H * p.ncta));
-    cfg.blockDim = dim3(kScanThreads);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

@@ -158,6 +158,17 @@ __device__ __forceinline__ void topk_weights(const uint64_t (&out)[KMAX], int K,
     }
 }
 
+// Gated Sparse Update, step 1 (retention): (1 - w)^(g/(1-g)) with the write gate g
+// clamped to [0,1] (NaN -> 0); 1 when w <= 0 or g == 0, 0 when w >= 1 or g == 1.
+__device__ __forceinline__ float gsu_alpha(float w, float g)
+{
+    g = fminf(fmaxf(g, 0.0f), 1.0f);
+    const float c = g / (1.0f - g);
+    if (w <= 0.0f || c <= 0.0f) return 1.0f;
+    if (w >= 1.0f) return 0.0f;
+    return expf(c * log1pf(-w));
+}
+
 // CAPE: (idx + pos) mod M, pos any 64-bit position.
 __device__ __forceinline__ int32_t cape_shift(int32_t idx, int64_t pos, int32_t M)
 {
