@@ -9,10 +9,19 @@
 // and, within one token, the K writes come before the K reads (the read sees the
 // token's own write).  Owners of one scan CTA are contiguous (o / 8 = CTA rank).
 //
-// Block = (b, h, chunk of C tokens); thread = (token, stream).  Each thread decodes one
-// address (stream 0: key -> writes, stream 1: query -> reads), then a stable counting
-// sort by owner places its K events: the owner-major table of per-thread counts is
-// exclusive-scanned once, which yields every event's position.
+// Each owner list is also cut into batches of at most 8 consecutive events on distinct
+// slots; the scan kernel loads a whole batch from tensor memory with one wait.
+//
+// Output per (b, h, chunk), one contiguous block of `chunk_bytes` (see ChunkLayout):
+//   offs[NO + 1]   start of each owner's segment, then the total event count
+//   recs[2*C*K]    {meta, weight}: meta = t << 16 | write << 15 | batch_len << 10 | column
+//                  (batch_len is set on the first event of each batch, 0 elsewhere)
+//   alph[2*C*K]    GSU retention of write events (0 for reads)
+//
+// Block = (b, h, G consecutive chunks of C tokens); thread = (chunk, stream, token).  Each
+// thread decodes one address (stream 0: key -> writes, stream 1: query -> reads); a
+// stable counting sort by owner (one exclusive scan of the chunk-major, owner-major count
+// table) places its K events within its chunk.
 #include "common.cuh"
 #include "kernels.h"
 #include "topk.cuh"
@@ -21,7 +30,7 @@ namespace ramnet {
 
 namespace {
 
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot)
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total_out)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
     int x = v;
@@ -32,12 +41,12 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot)
     }
     if (lane == 31) warp_tot[warp] = x;
     __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    int total = 0;
-    for (int w = 0; w < nw; ++w) total += warp_tot[w];
-    __syncthreads();
-    warp_tot[nw] = total;  // grand total (read after the caller's next barrier)
+    int base = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+        if (w < warp) base += warp_tot[w];
+        total += warp_tot[w];
+    }
+    *total_out = total;
     return base + x - v;
 }
 
@@ -45,18 +54,29 @@ template <int KMAX, int DPMAX>
 __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int C = p.chunk, nt = 2 * C;  // threads: stream-major (tid < C: key stream)
+    const int C = p.chunk, G = p.chunks_per_block;
+    const int nt = blockDim.x;         // whole warps; threads >= 2*C*G carry no token
+    const int nact = 2 * C * G;        // threads: (chunk g, stream, token)
     const int NO = 8 * p.ncta;
-    uint64_t* kept = reinterpret_cast<uint64_t*>(smem);                    // [KMAX][nt]
-    int* table = reinterpret_cast<int*>(smem + sizeof(uint64_t) * KMAX * nt);  // [NO][nt] counts -> positions
-    int* warp_tot = table + NO * nt;                                       // [nt/32 + 1]
+    const int E = 2 * C * p.K;         // event capacity of one chunk
+    const int TS = NO * 2 * C;         // table entries of one chunk
+    uint64_t* kept = reinterpret_cast<uint64_t*>(smem);                          // [KMAX][nt]
+    int* table = reinterpret_cast<int*>(smem + sizeof(uint64_t) * KMAX * nt);    // [G][NO][2C]
+    int* warp_tot = table + G * TS;                                              // [4]
+    uint2* srec = reinterpret_cast<uint2*>(warp_tot + 8);                        // [G][E]
+    float* salp = reinterpret_cast<float*>(srec + G * E);                        // [G][E]
+    int* soff = reinterpret_cast<int*>(salp + G * E);                            // [G][NO + 1]
 
-    const int bh = blockIdx.x / p.nchunks, c = blockIdx.x - bh * p.nchunks;
+    const int nblk = (p.nchunks + G - 1) / G;
+    const int bh = blockIdx.x / nblk, c0 = (blockIdx.x - bh * nblk) * G;
     const int b = bh / p.H, h = bh - b * p.H;
     const int tid = threadIdx.x;
-    const int stream = tid >= C ? 1 : 0, tl = tid - stream * C;
-    const int t0 = c * C, n = min(C, p.T - t0);
-    const bool valid = tl < n;
+    const bool active = tid < nact;
+    const int g = active ? tid / (2 * C) : 0, r2 = active ? tid - g * 2 * C : 0;
+    const int stream = r2 >= C ? 1 : 0, tl = r2 - stream * C;
+    const int c = c0 + g;
+    const int t0 = c * C, n = c < p.nchunks ? min(C, p.T - t0) : 0;
+    const bool valid = active && tl < n;
     const int so = 2 * tl + stream;  // position of this thread's events in token order
     const int L = p.U * p.d_p;
 
@@ -75,7 +95,7 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
         topk_weights<KMAX>(out, p.K, p.renorm, lg, th * L, p.in_bf16, p.d_p, p.U, w);
         const bool cape = p.cape_mask != nullptr && p.cape_mask[h] != 0;
         const int64_t pos = static_cast<int64_t>(p.pos0 != nullptr ? p.pos0[b] : 0) + t;
-        const float g = stream == 0 ? load_in(p.g, th, p.in_bf16) : 0.0f;
+        const float gg = stream == 0 ? load_in(p.g, th, p.in_bf16) : 0.0f;
         const int lg_ncta = __ffs(p.ncta) - 1;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
@@ -87,48 +107,93 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
                 meta[j] = (static_cast<uint32_t>(tl) << 16) | (stream == 0 ? 0x8000u : 0u) |
                           static_cast<uint32_t>((s >> 2) * p.cpl);
                 coef[j] = w[j];
-                alpha[j] = stream == 0 ? gsu_alpha(w[j], g) : 0.0f;
+                alpha[j] = stream == 0 ? gsu_alpha(w[j], gg) : 0.0f;
             }
         }
     }
 
-    // per-thread owner counts, owner-major: table[o * nt + so]
-    for (int i = tid; i < NO * nt; i += nt) table[i] = 0;
+    // per-thread owner counts: table[g][o][so]
+    int* tg = table + g * TS;
+    for (int i = tid; i < G * TS; i += nt) table[i] = 0;
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)
-        if (owner[j] >= 0) table[owner[j] * nt + so] += 1;
+        if (owner[j] >= 0) tg[owner[j] * 2 * C + so] += 1;
     __syncthreads();
-    // exclusive scan of the flattened table: thread i owns entries [i*NO, (i+1)*NO)
+    // exclusive scan of the flattened table (chunk-major, then owner, then token order);
+    // thread i owns entries [i*W, min((i+1)*W, G*TS)), W = ceil(G*TS / nt) <= NO
+    int total = 0;
     {
+        const int W = (G * TS + nt - 1) / nt;
+        const int lo = min(tid * W, G * TS), hi = min(lo + W, G * TS);
         int loc[64];
         int sum = 0;
-        for (int k = 0; k < NO; ++k) {
-            loc[k] = table[tid * NO + k];
+        for (int k = 0; k < hi - lo; ++k) {
+            loc[k] = table[lo + k];
             sum += loc[k];
         }
-        int run = block_exclusive_scan(sum, warp_tot);
-        for (int k = 0; k < NO; ++k) {
-            table[tid * NO + k] = run;
+        __syncthreads();
+        int run = block_exclusive_scan(sum, warp_tot, &total);
+        for (int k = 0; k < hi - lo; ++k) {
+            table[lo + k] = run;
             run += loc[k];
         }
     }
     __syncthreads();
-    // owner offsets of this chunk: start of each owner's segment, then the total
-    const long long chunk = static_cast<long long>(bh) * p.nchunks + c;
-    int* offs = p.offs + chunk * p.offs_stride;
-    for (int o = tid; o <= NO; o += nt) offs[o] = o < NO ? table[o * nt] : warp_tot[(nt + 31) / 32];
+    const int chunk_base = table[g * TS];  // read before the scatter below modifies the table
+    // per chunk: owner segment starts (relative to the chunk) and the chunk's total
+    for (int i = tid; i < G * (NO + 1); i += nt) {
+        const int gg = i / (NO + 1), o = i - gg * (NO + 1);
+        const int base = table[gg * TS];
+        const int next = gg + 1 < G ? table[(gg + 1) * TS] : total;
+        soff[i] = (o < NO ? table[gg * TS + o * 2 * C] : next) - base;
+    }
     __syncthreads();
-    // scatter: events of one owner keep token order (and writes before reads)
-    uint2* recs = p.recs + chunk * p.recs_stride;
-    float* alph = p.alphas + chunk * p.recs_stride;
+    // scatter into shared memory: events of one owner keep token order, writes first
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
         if (owner[j] >= 0) {
-            const int posn = table[owner[j] * nt + so];
-            table[owner[j] * nt + so] = posn + 1;
-            recs[posn] = make_uint2(meta[j], __float_as_uint(coef[j]));
-            alph[posn] = alpha[j];
+            const int posn = tg[owner[j] * 2 * C + so];
+            tg[owner[j] * 2 * C + so] = posn + 1;
+            srec[g * E + posn - chunk_base] = make_uint2(meta[j], __float_as_uint(coef[j]));
+            salp[g * E + posn - chunk_base] = alpha[j];
+        }
+    }
+    __syncthreads();
+    // batches: greedy runs of at most 8 events with distinct columns, per owner list
+    for (int i0 = tid; i0 < G * NO; i0 += nt) {
+        const int gg = i0 / NO, o = i0 - gg * NO;
+        uint2* rr = srec + gg * E;
+        int i = soff[gg * (NO + 1) + o];
+        const int end = soff[gg * (NO + 1) + o + 1];
+        while (i < end) {
+            uint32_t cols[8];
+            int nb = 0;
+            while (nb < 8 && i + nb < end) {
+                const uint32_t col = rr[i + nb].x & 0x3FFu;
+                bool dup = false;
+                for (int k = 0; k < nb; ++k) dup |= cols[k] == col;
+                if (dup) break;
+                cols[nb++] = col;
+            }
+            rr[i].x |= static_cast<uint32_t>(nb) << 10;
+            i += nb;
+        }
+    }
+    __syncthreads();
+    // the chunk blocks: offsets, records, retentions
+    for (int gg = 0; gg < G; ++gg) {
+        const int cc = c0 + gg;
+        if (cc >= p.nchunks) break;
+        unsigned char* blk = p.blocks + (static_cast<size_t>(bh) * p.nchunks + cc) * p.chunk_bytes;
+        int* goff = reinterpret_cast<int*>(blk);
+        uint2* grec = reinterpret_cast<uint2*>(blk + p.recs_off);
+        float* galp = reinterpret_cast<float*>(blk + p.alph_off);
+        const int cnt = soff[gg * (NO + 1) + NO];
+        for (int o = tid; o <= NO; o += nt) goff[o] = soff[gg * (NO + 1) + o];
+        for (int i = tid; i < cnt; i += nt) {
+            grec[i] = srec[gg * E + i];
+            galp[i] = salp[gg * E + i];
         }
     }
 }
@@ -136,13 +201,18 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
 template <int KMAX, int DPMAX>
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s)
 {
-    const int nt = 2 * p.chunk;
+    const int G = p.chunks_per_block;
+    const int nt = 2 * p.chunk * G;
     const int NO = 8 * p.ncta;
-    const size_t smem = sizeof(uint64_t) * KMAX * nt + sizeof(int) * (NO * nt + nt / 32 + 2);
+    const int E = 2 * p.chunk * p.K;
+    const size_t smem = sizeof(uint64_t) * KMAX * ((nt + 31) / 32 * 32) + sizeof(int) * (G * NO * 2 * p.chunk + 8) +
+                        (sizeof(uint2) + sizeof(float)) * G * E + sizeof(int) * G * (NO + 1);
     auto kern = k_decode_route<KMAX, DPMAX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(p.B * p.H * p.nchunks), nt, smem, s>>>(p);
+    const int nblk = (p.nchunks + G - 1) / G;
+    const int threads = (nt + 31) / 32 * 32;  // whole warps (the block scan uses full-warp shuffles)
+    kern<<<static_cast<unsigned>(p.B * p.H * nblk), threads, smem, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -157,9 +227,13 @@ cudaError_t route_k(const RouteParams& p, cudaStream_t s)
 
 }  // namespace
 
-cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream)
+cudaError_t launch_decode_route(const RouteParams& p_in, cudaStream_t stream)
 {
+    RouteParams p = p_in;
     if (2 * p.chunk > 128 || 8 * p.ncta > 64) return cudaErrorInvalidValue;
+    // as many chunks per block as fit 128 threads, keeping the flattened table divisible
+    p.chunks_per_block = 1;
+    while (2 * p.chunk * p.chunks_per_block * 2 <= 128 && p.chunks_per_block * 2 <= p.nchunks) p.chunks_per_block *= 2;
     if (p.d_p <= 4) return route_k<4>(p, stream);
     if (p.d_p <= 8) return route_k<8>(p, stream);
     return route_k<16>(p, stream);

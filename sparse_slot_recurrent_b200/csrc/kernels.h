@@ -23,6 +23,9 @@ struct DecodeParams {
 
 // Decode + route (first kernel of the prefill scan): per (b, h, chunk) the token-ordered
 // event list of every owner warp of the scan kernel.
+// Decode + route (first kernel of the prefill scan): per (b, h, chunk) one block of
+// `chunk_bytes` holding the owner offsets, the owner-sorted event records and the write
+// retentions (layout: chunk_block_bytes()).
 struct RouteParams {
     const void* k_logits;  // [B,T,H,U*d_p]
     const void* q_logits;
@@ -33,21 +36,16 @@ struct RouteParams {
     const int32_t* pos0;       // [B] or null
     const uint8_t* cape_mask;  // [H] or null
     int ncta, cpl, chunk, nchunks;
-    uint2* recs;      // [B*H*nchunks][recs_stride] {meta, weight}
-    float* alphas;    // same indexing: GSU retention of write events
-    long long recs_stride;
-    int* offs;        // [B*H*nchunks][offs_stride]: owner segment starts, then the total
-    long long offs_stride;
+    int chunks_per_block;   // set by the launcher
+    unsigned char* blocks;  // [B*H*nchunks][chunk_bytes]
+    size_t chunk_bytes, recs_off, alph_off;
 };
 
 struct ScanParams {
-    const uint2* recs;
-    const float* alphas;
-    long long recs_stride;
-    const int* offs;
-    long long offs_stride;
-    const void* v;        // [B,T,H,d_v]
-    const void* z;        // [B,T,H,d_v]
+    const unsigned char* blocks;  // chunk blocks written by the route kernel
+    size_t chunk_bytes, recs_off, alph_off;
+    const void* v;  // [B,T,H,d_v]
+    const void* z;  // [B,T,H,d_v]
     int in_bf16;
     const float* norm_w;  // [d_v] or null
     const float* S_in;    // [B,H,M,d_v] or null
@@ -92,6 +90,8 @@ struct StepParams {
 // slot array, the chunk length, and the TMEM columns and shared memory of each CTA.
 // Returns false if the slot array does not fit.
 bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* plan);
+// Bytes of one chunk block (offsets, records, retentions) and the offsets of its parts.
+size_t chunk_block_bytes(int chunk, int K, int ncta, size_t* recs_off, size_t* alph_off);
 
 cudaError_t launch_decode_addresses(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream);

@@ -80,27 +80,19 @@ uint32_t* device_status_ptr()
     return static_cast<uint32_t*>(p);
 }
 
-// Scratch of the prefill scan: per (b, h, chunk) the owner-sorted event records, the
-// retention of each write event, and the owner offsets.
+// Scratch of the prefill scan: one block per (b, h, chunk) with the owner offsets, the
+// owner-sorted event records and the write retentions, plus padding for bulk copies.
 struct WorkspaceLayout {
-    size_t recs, alphas, offs, total;
-    long long recs_stride, offs_stride;
+    size_t chunk_bytes, recs_off, alph_off, total;
     int nchunks;
 };
-
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 WorkspaceLayout workspace_layout(int B, int T, int H, int K, const ramnet::ScanPlan& plan)
 {
     WorkspaceLayout w;
     w.nchunks = (T + plan.chunk - 1) / plan.chunk;
-    w.recs_stride = static_cast<long long>(round_up(static_cast<size_t>(2 * plan.chunk * K), 4));
-    w.offs_stride = static_cast<long long>(round_up(static_cast<size_t>(8 * plan.ncta + 1), 4));
-    const size_t n = static_cast<size_t>(B) * H * w.nchunks;
-    w.recs = 0;
-    w.alphas = round_up(w.recs + n * w.recs_stride * sizeof(uint2) + 256, 256);
-    w.offs = round_up(w.alphas + n * w.recs_stride * sizeof(float) + 256, 256);
-    w.total = round_up(w.offs + n * w.offs_stride * sizeof(int) + 256, 256);
+    w.chunk_bytes = ramnet::chunk_block_bytes(plan.chunk, K, plan.ncta, &w.recs_off, &w.alph_off);
+    w.total = static_cast<size_t>(B) * H * w.nchunks * w.chunk_bytes + 256;
     return w;
 }
 
@@ -176,7 +168,6 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
         return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, wl.total);
     uint32_t* status = device_status_ptr();
     if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-    char* ws = static_cast<char*>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     ramnet::RouteParams rp{};
@@ -198,20 +189,18 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     rp.cpl = plan.cpl;
     rp.chunk = plan.chunk;
     rp.nchunks = wl.nchunks;
-    rp.recs = reinterpret_cast<uint2*>(ws + wl.recs);
-    rp.alphas = reinterpret_cast<float*>(ws + wl.alphas);
-    rp.recs_stride = wl.recs_stride;
-    rp.offs = reinterpret_cast<int*>(ws + wl.offs);
-    rp.offs_stride = wl.offs_stride;
+    rp.blocks = static_cast<unsigned char*>(workspace);
+    rp.chunk_bytes = wl.chunk_bytes;
+    rp.recs_off = wl.recs_off;
+    rp.alph_off = wl.alph_off;
     cudaError_t e = ramnet::launch_decode_route(rp, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan: decode/route launch");
 
     ramnet::ScanParams sp{};
-    sp.recs = rp.recs;
-    sp.alphas = rp.alphas;
-    sp.recs_stride = wl.recs_stride;
-    sp.offs = rp.offs;
-    sp.offs_stride = wl.offs_stride;
+    sp.blocks = rp.blocks;
+    sp.chunk_bytes = wl.chunk_bytes;
+    sp.recs_off = wl.recs_off;
+    sp.alph_off = wl.alph_off;
     sp.v = v;
     sp.z = z;
     sp.in_bf16 = in_dt == RAMNET_BF16;

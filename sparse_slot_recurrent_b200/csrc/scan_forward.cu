@@ -14,17 +14,22 @@
 // them their write masses (shared memory).
 //
 // Work per chunk of C tokens (the decode kernel has already sorted the chunk's events
-// into one token-ordered list per owner warp):
-//   loader warp    bulk-copies this CTA's lists, the write retentions and the chunk's
-//                  value rows into shared memory (2-deep ring);
-//   scan warps     walk their own list in batches of up to 4 events on distinct slots:
-//                  one tcgen05.ld per event, one wait, then writes (mass, rate, content)
-//                  and reads (weighted row red-added into the chunk's o buffer);
-//   epilogue warps add the partial o of all CTAs of the cluster through distributed
-//                  shared memory, exchange the squared norms the same way, and write
-//                  y = o / rms(o) * norm_w * z for this CTA's share of the channels.
+// into one token-ordered list per owner warp, cut into batches on distinct slots):
+//   loader warp    bulk-copies the chunk block (owner offsets, event records, write
+//                  retentions), the chunk's value rows and this CTA's output-gate
+//                  columns into a ring of shared-memory stages;
+//   scan warps     walk their own list one batch at a time: one tcgen05.ld per event and
+//                  one wait per batch; writes update mass, rate and content; reads are
+//                  summed in registers per token and stored once per (warp, token) as a
+//                  partial row plus a flag byte;
+//   epilogue warps (a) add up a chunk's partial rows and push the sum to every CTA of
+//                  the cluster (stores into the peers' shared memory), (b) kLag chunks
+//                  later add the pushed sums of all CTAs, apply RMSNorm over d_v and the
+//                  output gate, and store y for this CTA's share of the channels.  The
+//                  lag hides the latency of the cross-SM exchange.
 // Every hand-off is an mbarrier; every wait is bounded (about 2 s); a wait that gives up
-// records RAMNET_ERR_TIMEOUT in the status word and the kernel carries on to the end.
+// records RAMNET_ERR_TIMEOUT in the status word, raises the CTA's abort flag and the
+// kernel carries on to the end without further waiting.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -37,45 +42,54 @@ constexpr int kLoadWarp = 8;
 constexpr int kEpiWarp0 = 9;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = (kScanWarps + 1 + kEpiWarps) * 32;
+constexpr int kStages = 6;  // staging ring depth
+constexpr int kLag = 2;     // the epilogue finishes chunk c - kLag after pushing chunk c
+// ring of pushed sums: a CTA may push chunk d + kRecv into a peer only after that peer has
+// finished chunk d; with the push of chunk c issued before finishing chunk c - kLag this
+// needs kRecv >= 2 * kLag + 2
+constexpr int kRecv = 2 * kLag + 2;
 
-enum Bar { kStage = 0, kScan = 2, kOFree = 4, kZ = 6, kPeerO = 8, kPeerSS = 10, kFin = 12, kNumBars = 13 };
+// mbarrier indices
+constexpr int kBarStage = 0;                           // [kStages] staged data landed (tx)
+constexpr int kBarStageFree = kBarStage + kStages;     // [kStages] scan + epilogue done with a stage
+constexpr int kBarRowsFull = kBarStageFree + kStages;  // [2] scan warps done with a chunk
+constexpr int kBarRowsFree = kBarRowsFull + 2;         // [2] epilogue consumed the partial rows
+constexpr int kBarRecv = kBarRowsFree + 2;             // [kRecv] every CTA pushed its sums
+constexpr int kBarFin = kBarRecv + kRecv;
+constexpr int kNumBars = kBarFin + 1;
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 struct Layout {
-    size_t bars, holder, m, offs, recs, alph, vbuf, zbuf, obuf, ss, total;
-    size_t recs_bytes, alph_bytes, vbuf_bytes, zbuf_bytes, obuf_bytes;
+    size_t bars, misc, m, stage, rows, flags, recv, total;
+    size_t stage_bytes, blk_bytes, v_off, z_off, rows_bytes, flags_bytes, recv_bytes;
 };
 
-__host__ __device__ inline Layout scan_layout(int Ml, int C, int K, int dv, int ncta, int es)
+__host__ __device__ inline Layout scan_layout(int Ml, int C, int dv, int ncta, int es, size_t chunk_bytes)
 {
     Layout L;
-    L.recs_bytes = align16(sizeof(uint2) * (2 * C * K + 4));
-    L.alph_bytes = align16(sizeof(float) * (2 * C * K + 8));
-    L.vbuf_bytes = align16(static_cast<size_t>(C) * dv * es);
-    L.zbuf_bytes = align16(static_cast<size_t>(C) * (dv / ncta) * es);
-    L.obuf_bytes = align16(sizeof(float) * C * dv);
+    L.blk_bytes = align16(chunk_bytes);
+    L.v_off = L.blk_bytes;
+    L.z_off = L.v_off + align16(static_cast<size_t>(C) * dv * es);
+    L.stage_bytes = L.z_off + align16(static_cast<size_t>(C) * (dv / ncta) * es);
+    L.rows_bytes = align16(sizeof(float) * C * kScanWarps * dv);
+    L.flags_bytes = align16(static_cast<size_t>(C) * kScanWarps);
+    L.recv_bytes = align16(sizeof(float) * ncta * C * dv);
     size_t o = 0;
     L.bars = o;
     o += align16(8 * kNumBars);
-    L.holder = o;
+    L.misc = o;
     o += 16;
-    L.offs = o;  // per buffer: 9 owner offsets + record base + alpha base
-    o += align16(sizeof(int) * 2 * 12);
     L.m = o;
     o += align16(sizeof(float) * Ml);
-    L.recs = o;
-    o += 2 * L.recs_bytes;
-    L.alph = o;
-    o += 2 * L.alph_bytes;
-    L.vbuf = o;
-    o += 2 * L.vbuf_bytes;
-    L.zbuf = o;
-    o += 2 * L.zbuf_bytes;
-    L.obuf = o;
-    o += 2 * L.obuf_bytes;
-    L.ss = o;
-    o += align16(sizeof(float) * 2 * C);
+    L.stage = o;
+    o += kStages * L.stage_bytes;
+    L.rows = o;
+    o += 2 * L.rows_bytes;
+    L.flags = o;
+    o += 2 * L.flags_bytes;
+    L.recv = o;
+    o += kRecv * L.recv_bytes;
     L.total = o;
     return L;
 }
@@ -163,10 +177,18 @@ __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.
 
 __device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); }
 
-// Cluster-wide signal: one thread arrives on the same mbarrier of every CTA.
-__device__ __forceinline__ void signal_cluster(uint32_t bar, int ncta)
+// 16-byte store into the shared memory of cluster CTA `rank` (same offset as `local`).
+__device__ __forceinline__ void st_cluster_v4(const void* local, uint32_t rank, float4 v)
 {
-    for (int r = 0; r < ncta; ++r) mbar_arrive_cluster(map_to_rank(bar, static_cast<uint32_t>(r)));
+    const uint32_t a = map_to_rank(smem_addr(local), rank);
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_f32(const void* local, uint32_t rank, float v)
+{
+    const uint32_t a = map_to_rank(smem_addr(local), rank);
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
 
 // CPL consecutive input elements (fp32 or bf16) from shared memory, as fp32.
@@ -175,12 +197,59 @@ __device__ __forceinline__ void load_row(const unsigned char* base, int elem, in
 {
     if (is_bf16) {
         const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(base) + elem;
+        if constexpr (CPL % 4 == 0) {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) v[c] = __bfloat162float(pb[c]);
+            for (int c = 0; c < CPL; c += 4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(pb + c);
+                v[c + 0] = __uint_as_float(u.x << 16);
+                v[c + 1] = __uint_as_float(u.x & 0xFFFF0000u);
+                v[c + 2] = __uint_as_float(u.y << 16);
+                v[c + 3] = __uint_as_float(u.y & 0xFFFF0000u);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) v[c] = __bfloat162float(pb[c]);
+        }
     } else {
         const float* pf = reinterpret_cast<const float*>(base) + elem;
+        if constexpr (CPL % 4 == 0) {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) v[c] = pf[c];
+            for (int c = 0; c < CPL; c += 4) {
+                const float4 u = *reinterpret_cast<const float4*>(pf + c);
+                v[c] = u.x;
+                v[c + 1] = u.y;
+                v[c + 2] = u.z;
+                v[c + 3] = u.w;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) v[c] = pf[c];
+        }
+    }
+}
+
+template <int CPL>
+__device__ __forceinline__ void store_row(float* dst, const float (&v)[CPL])
+{
+    if constexpr (CPL % 4 == 0) {
+#pragma unroll
+        for (int c = 0; c < CPL; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+    } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) dst[c] = v[c];
+    }
+}
+
+// Push CPL values to the same location in cluster CTA `rank`.
+template <int CPL>
+__device__ __forceinline__ void push_row(float* dst, uint32_t rank, const float (&v)[CPL])
+{
+    if constexpr (CPL % 4 == 0) {
+#pragma unroll
+        for (int c = 0; c < CPL; c += 4) st_cluster_v4(dst + c, rank, make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
+    } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) st_cluster_f32(dst + c, rank, v[c]);
     }
 }
 
@@ -198,33 +267,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Ml = (M - static_cast<int>(rank) + ncta - 1) / ncta;
     const int nch = (p.T + C - 1) / C;
-    const Layout L = scan_layout((M + ncta - 1) / ncta, C, p.K, dv, ncta, es);
+    const Layout L = scan_layout((M + ncta - 1) / ncta, C, dv, ncta, es, p.chunk_bytes);
     const uint32_t bars = smem_addr(smem + L.bars);
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-    uint32_t* holder = reinterpret_cast<uint32_t*>(smem + L.holder);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.holder + 4);
-    int* offs_s = reinterpret_cast<int*>(smem + L.offs);
+    uint64_t* bar_ptr = reinterpret_cast<uint64_t*>(smem + L.bars);
+    uint32_t* holder = reinterpret_cast<uint32_t*>(smem + L.misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
     float* m_s = reinterpret_cast<float*>(smem + L.m);
-    float* ss_s = reinterpret_cast<float*>(smem + L.ss);
+    auto stage = [&](int c) { return smem + L.stage + static_cast<size_t>(c % kStages) * L.stage_bytes; };
 
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kStage + i, 1);
-            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kScan + i, kScanWarps * 32);
-            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kOFree + i, kEpiWarps * 32);
-            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kZ + i, 1);
-            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kPeerO + i, static_cast<uint32_t>(ncta));
-            mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kPeerSS + i, static_cast<uint32_t>(ncta));
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(bar_ptr + kBarStage + i, 1);
+            mbar_init(bar_ptr + kBarStageFree + i, (kScanWarps + kEpiWarps) * 32);
         }
-        mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars) + kFin, static_cast<uint32_t>(ncta));
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_ptr + kBarRowsFull + i, kScanWarps * 32);
+            mbar_init(bar_ptr + kBarRowsFree + i, kEpiWarps * 32);
+        }
+        for (int i = 0; i < kRecv; ++i) mbar_init(bar_ptr + kBarRecv + i, static_cast<uint32_t>(ncta));
+        mbar_init(bar_ptr + kBarFin, static_cast<uint32_t>(ncta));
         fence_mbar_init_cluster();
     }
     if (warp == 0) tmem_alloc(holder, p.tmem_cols);
-    // zero both o buffers and the masses / initial state
     {
-        float4* ob = reinterpret_cast<float4*>(smem + L.obuf);
-        for (size_t i = tid; i < 2 * L.obuf_bytes / 16; i += kThreads) ob[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        uint32_t* fl = reinterpret_cast<uint32_t*>(smem + L.flags);
+        for (size_t i = tid; i < 2 * L.flags_bytes / 4; i += kThreads) fl[i] = 0u;
         for (int s = tid; s < Ml; s += kThreads)
             m_s[s] = p.m_in != nullptr ? p.m_in[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] : 0.0f;
     }
@@ -238,63 +307,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
         // ============================================================ scan warps
         const int q = warp & 3;
         const uint32_t tq = tbase + (static_cast<uint32_t>(32 * q) << 16);
+        const int lch = (lane < LW ? lane : 0) * CPL;  // this lane's first channel
         for (int s = warp; s < Ml; s += 8) {
             const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
             float r[CPL];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) r[c] = (p.S_in != nullptr && lane < LW) ? p.S_in[row + lane * CPL + c] : 0.0f;
+            for (int c = 0; c < CPL; ++c) r[c] = (p.S_in != nullptr && lane < LW) ? p.S_in[row + lch + c] : 0.0f;
             tmem_st<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), r);
         }
         tmem_wait_st();
         for (int c = 0; c < nch; ++c) {
-            const int bf = c & 1;
-            wait_bounded<false>(bar(kStage + bf), (c >> 1) & 1, p.status, abort_flag);
-            if (c >= 2) wait_bounded<false>(bar(kOFree + bf), ((c - 2) >> 1) & 1, p.status, abort_flag);
-            const uint2* recs = reinterpret_cast<const uint2*>(smem + L.recs + bf * L.recs_bytes);
-            const float* alph = reinterpret_cast<const float*>(smem + L.alph + bf * L.alph_bytes);
-            const unsigned char* vb = smem + L.vbuf + bf * L.vbuf_bytes;
-            float* ob = reinterpret_cast<float*>(smem + L.obuf + bf * L.obuf_bytes);
-            const int* ofs = offs_s + bf * 12;
-            const int rbase = ofs[9], abase = ofs[10];
-            const int end = ofs[warp + 1] - rbase;
-            const int ashift = rbase - abase;
-            for (int i = ofs[warp] - rbase; i < end;) {
-                // a batch of up to 4 events on distinct slots (columns)
-                uint2 r[4];
-                r[0] = recs[i];
-                int nb = 1;
-                if (i + 1 < end) {
-                    r[1] = recs[i + 1];
-                    const uint32_t c0 = r[0].x & 0x7FFFu, c1 = r[1].x & 0x7FFFu;
-                    if (c1 != c0) {
-                        nb = 2;
-                        if (i + 2 < end) {
-                            r[2] = recs[i + 2];
-                            const uint32_t c2 = r[2].x & 0x7FFFu;
-                            if (c2 != c0 && c2 != c1) {
-                                nb = 3;
-                                if (i + 3 < end) {
-                                    r[3] = recs[i + 3];
-                                    const uint32_t c3 = r[3].x & 0x7FFFu;
-                                    if (c3 != c0 && c3 != c1 && c3 != c2) nb = 4;
-                                }
-                            }
-                        }
-                    }
-                }
-                float S[4][CPL];
+            const int rb = c & 1;
+            wait_bounded<false>(bar(kBarStage + c % kStages), (c / kStages) & 1, p.status, abort_flag);
+            if (c >= 2) wait_bounded<false>(bar(kBarRowsFree + rb), ((c - 2) >> 1) & 1, p.status, abort_flag);
+            const unsigned char* st = stage(c);
+            const int* ofs = reinterpret_cast<const int*>(st);
+            const uint2* recs = reinterpret_cast<const uint2*>(st + p.recs_off);
+            const float* alph = reinterpret_cast<const float*>(st + p.alph_off);
+            const unsigned char* vb = st + L.v_off;
+            float* rows = reinterpret_cast<float*>(smem + L.rows + rb * L.rows_bytes);
+            unsigned char* flags = smem + L.flags + rb * L.flags_bytes;
+            const int o = static_cast<int>(rank) * 8 + warp;
+            int i = ofs[o];
+            const int end = ofs[o + 1];
+            int cur_t = -1;  // token whose read sum is being accumulated
+            float acc[CPL];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (k < nb) tmem_ld<CPL>(tq + (r[k].x & 0x7FFFu), S[k]);
+            for (int cc = 0; cc < CPL; ++cc) acc[cc] = 0.0f;
+            while (i < end) {
+                const int nb = static_cast<int>((recs[i].x >> 10) & 0xFu);
+                uint2 r[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) r[k] = k < nb ? recs[i + k] : make_uint2(0u, 0u);
+                float S[8][CPL];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < nb) tmem_ld<CPL>(tq + (r[k].x & 0x3FFu), S[k]);
                 // masses and rates of the batch's writes while the loads are in flight
-                float lam[4];
+                float lam[8];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                for (int k = 0; k < 8; ++k) {
                     lam[k] = 0.0f;
                     if (k < nb && (r[k].x & 0x8000u)) {
-                        const int s = 4 * static_cast<int>((r[k].x & 0x7FFFu) / CPL) + q;
+                        const int s = 4 * static_cast<int>((r[k].x & 0x3FFu) / CPL) + q;
                         const float w = __uint_as_float(r[k].y);
-                        const float mn = alph[i + k + ashift] * m_s[s] + w;
+                        const float mn = alph[i + k] * m_s[s] + w;
                         lam[k] = w * __frcp_rn(mn + p.eps_gsu);
                         __syncwarp();
                         if (lane == 0) m_s[s] = mn;
@@ -302,27 +359,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
                 }
                 __syncwarp();
                 tmem_wait_ld();
+                bool any_write = false;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                for (int k = 0; k < 8; ++k) {
                     if (k < nb) {
                         const int t = static_cast<int>(r[k].x >> 16);
                         if (r[k].x & 0x8000u) {
                             float vv[CPL];
-                            load_row<CPL>(vb, t * dv + (lane < LW ? lane : 0) * CPL, p.in_bf16, vv);
+                            load_row<CPL>(vb, t * dv + lch, p.in_bf16, vv);
 #pragma unroll
                             for (int cc = 0; cc < CPL; ++cc) S[k][cc] = fmaf(lam[k], vv[cc] - S[k][cc], S[k][cc]);
-                            tmem_st<CPL>(tq + (r[k].x & 0x7FFFu), S[k]);
-                        } else if (lane < LW) {
+                            tmem_st<CPL>(tq + (r[k].x & 0x3FFu), S[k]);
+                            any_write = true;
+                        } else {
+                            if (t != cur_t) {
+                                if (cur_t >= 0) {
+                                    if (lane < LW) store_row<CPL>(rows + (cur_t * kScanWarps + warp) * dv + lch, acc);
+                                    if (lane == 0) flags[cur_t * kScanWarps + warp] = 1;
+                                }
+                                cur_t = t;
+#pragma unroll
+                                for (int cc = 0; cc < CPL; ++cc) acc[cc] = 0.0f;
+                            }
                             const float rw = __uint_as_float(r[k].y);
 #pragma unroll
-                            for (int cc = 0; cc < CPL; ++cc) atomicAdd(&ob[t * dv + cc * LW + lane], rw * S[k][cc]);
+                            for (int cc = 0; cc < CPL; ++cc) acc[cc] = fmaf(rw, S[k][cc], acc[cc]);
                         }
                     }
                 }
-                tmem_wait_st();
+                if (any_write) tmem_wait_st();
                 i += nb;
             }
-            arrive_cta(bar(kScan + bf));
+            if (cur_t >= 0) {
+                if (lane < LW) store_row<CPL>(rows + (cur_t * kScanWarps + warp) * dv + lch, acc);
+                if (lane == 0) flags[cur_t * kScanWarps + warp] = 1;
+            }
+            arrive_cta(bar(kBarRowsFull + rb));
+            arrive_cta(bar(kBarStageFree + c % kStages));
         }
         // final state of the owned slots
         for (int s = warp; s < Ml; s += 8) {
@@ -332,144 +405,137 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             tmem_wait_ld();
             if (lane < LW) {
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) p.S_out[row + lane * CPL + c] = r[c];
+                for (int c = 0; c < CPL; ++c) p.S_out[row + lch + c] = r[c];
             }
             if (lane == 0) p.m_out[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] = m_s[s];
         }
     } else if (warp == kLoadWarp) {
         // ============================================================ loader warp
+        const uint32_t vrow = static_cast<uint32_t>(dv * es);
+        const uint32_t zrow = static_cast<uint32_t>(Dr * es);
+        const uint32_t blk = static_cast<uint32_t>(p.chunk_bytes);
         for (int c = 0; c < nch; ++c) {
-            const int bf = c & 1;
             const int n = min(C, p.T - c * C);
-            if (c >= 2) {
-                wait_bounded<false>(bar(kScan + bf), ((c - 2) >> 1) & 1, p.status, abort_flag);
+            if (c >= kStages) {
+                wait_bounded<false>(bar(kBarStageFree + c % kStages), (c / kStages - 1) & 1, p.status, abort_flag);
                 fence_proxy_async();
             }
-            const long long chunk = static_cast<long long>(bh) * nch + c;
-            const int* og = p.offs + chunk * p.offs_stride + 8 * rank;
-            const int o = lane < 9 ? og[lane] : 0;
-            const int lo = __shfl_sync(0xffffffffu, o, 0), hi = __shfl_sync(0xffffffffu, o, 8);
-            const int lo_r = lo & ~1, lo_a = lo & ~3;
-            const uint32_t rb = hi > lo ? static_cast<uint32_t>(align16(static_cast<size_t>(hi - lo_r) * 8)) : 0u;
-            const uint32_t ab = hi > lo ? static_cast<uint32_t>(align16(static_cast<size_t>(hi - lo_a) * 4)) : 0u;
-            const uint32_t vrow = static_cast<uint32_t>(dv * es);
-            int* ofs = offs_s + bf * 12;
-            if (lane < 9) ofs[lane] = o;
-            if (lane == 9) ofs[9] = lo_r;
-            if (lane == 10) ofs[10] = lo_a;
+            unsigned char* st = stage(c);
+            const uint32_t sb = bar(kBarStage + c % kStages);
+            if (lane == 0) arrive_expect_tx(sb, blk + static_cast<uint32_t>(n) * (vrow + zrow));
             __syncwarp();
-            if (lane == 0) arrive_expect_tx(bar(kStage + bf), rb + ab + static_cast<uint32_t>(n) * vrow);
-            __syncwarp();
-            if (lane == 0 && rb) bulk_g2s(smem_addr(smem + L.recs + bf * L.recs_bytes), p.recs + chunk * p.recs_stride + lo_r, rb, bar(kStage + bf));
-            if (lane == 1 && ab) bulk_g2s(smem_addr(smem + L.alph + bf * L.alph_bytes), p.alphas + chunk * p.recs_stride + lo_a, ab, bar(kStage + bf));
+            if (lane == 0)
+                bulk_g2s(smem_addr(st), p.blocks + (static_cast<size_t>(bh) * nch + c) * p.chunk_bytes, blk, sb);
             for (int t = lane; t < n; t += 32) {
                 const size_t th = (static_cast<size_t>(b) * p.T + c * C + t) * p.H + h;
-                bulk_g2s(smem_addr(smem + L.vbuf + bf * L.vbuf_bytes + static_cast<size_t>(t) * vrow),
-                         static_cast<const unsigned char*>(p.v) + th * vrow, vrow, bar(kStage + bf));
+                bulk_g2s(smem_addr(st + L.v_off + static_cast<size_t>(t) * vrow),
+                         static_cast<const unsigned char*>(p.v) + th * vrow, vrow, sb);
+                bulk_g2s(smem_addr(st + L.z_off + static_cast<size_t>(t) * zrow),
+                         static_cast<const unsigned char*>(p.z) + (th * dv + static_cast<size_t>(rank) * Dr) * es, zrow, sb);
             }
         }
     } else {
         // ============================================================ epilogue warps
         const int e = warp - kEpiWarp0;
-        const int etid = tid - kEpiWarp0 * 32;
-        const int cpl_lane = Dr >= 32 ? Dr / 32 : 1;  // output channels per lane
-        const bool lane_on = lane * cpl_lane < Dr;
-        const int ch0 = static_cast<int>(rank) * Dr + lane * cpl_lane;
-        const uint32_t zrow = static_cast<uint32_t>(Dr * es);
-        for (int c = 0; c < nch; ++c) {
-            const int bf = c & 1;
-            const int n = min(C, p.T - c * C);
-            const int t0 = c * C;
-            // stage z (this CTA's channels) for the chunk
-            if (e == 0) {
-                fence_proxy_async();
-                if (lane == 0) arrive_expect_tx(bar(kZ + bf), static_cast<uint32_t>(n) * zrow);
-                __syncwarp();
-                for (int t = lane; t < n; t += 32) {
-                    const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
-                    bulk_g2s(smem_addr(smem + L.zbuf + bf * L.zbuf_bytes + static_cast<size_t>(t) * zrow),
-                             static_cast<const unsigned char*>(p.z) + (th * dv + static_cast<size_t>(rank) * Dr) * es,
-                             zrow, bar(kZ + bf));
-                }
-            }
-            wait_bounded<false>(bar(kScan + bf), (c >> 1) & 1, p.status, abort_flag);
-            float* ob = reinterpret_cast<float*>(smem + L.obuf + bf * L.obuf_bytes);
-            float* ss = ss_s + bf * C;
-            // all CTAs' partial sums of this chunk are complete
-            if (etid == 0) {
-                if (ncta == 1) arrive_cta(bar(kPeerO + bf));
-                else signal_cluster(bar(kPeerO + bf), ncta);
-            }
-            wait_bounded<true>(bar(kPeerO + bf), (c >> 1) & 1, p.status, abort_flag);
-            for (int t = e; t < n; t += kEpiWarps) {
-                float sq = 0.0f;
-                if (lane_on) {
-                    for (int k = 0; k < cpl_lane; ++k) {
-                        const int ch = ch0 + k;
-                        const int pos = t * dv + (ch % CPL) * LW + ch / CPL;
-                        float o = 0.0f;
-                        if (ncta == 1) {
-                            o = ob[pos];
-                        } else {
-                            const uint32_t a = smem_addr(&ob[pos]);
-                            for (int r = 0; r < ncta; ++r) o += ld_cluster_f32(map_to_rank(a, static_cast<uint32_t>(r)));
-                            ob[pos] = o;
-                        }
-                        sq += o * o;
-                    }
-                }
+        const int lch = (lane < LW ? lane : 0) * CPL;
+        const bool mine = lane < LW && lch >= static_cast<int>(rank) * Dr && lch < (static_cast<int>(rank) + 1) * Dr;
+        float nw[CPL];
 #pragma unroll
-                for (int d = 16; d > 0; d >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, d);
-                if (lane == 0) ss[t] = sq;
-            }
-            epi_barrier();
-            if (etid == 0) {
-                if (ncta == 1) arrive_cta(bar(kPeerSS + bf));
-                else signal_cluster(bar(kPeerSS + bf), ncta);
-            }
-            wait_bounded<true>(bar(kPeerSS + bf), (c >> 1) & 1, p.status, abort_flag);
-            wait_bounded<false>(bar(kZ + bf), (c >> 1) & 1, p.status, abort_flag);
-            const unsigned char* zb = smem + L.zbuf + bf * L.zbuf_bytes;
-            for (int t = e; t < n; t += kEpiWarps) {
-                float tot = 0.0f;
-                if (ncta == 1) {
-                    tot = ss[t];
-                } else {
-                    const uint32_t a = smem_addr(&ss[t]);
-                    for (int r = 0; r < ncta; ++r) tot += ld_cluster_f32(map_to_rank(a, static_cast<uint32_t>(r)));
+        for (int cc = 0; cc < CPL; ++cc) nw[cc] = p.norm_w != nullptr ? p.norm_w[lch + cc] : 1.0f;
+        for (int c = 0; c < nch + kLag; ++c) {
+            // (a) chunk c: sum this CTA's partial rows and push them to every CTA
+            if (c < nch) {
+                const int rb = c & 1;
+                const int n = min(C, p.T - c * C);
+                wait_bounded<false>(bar(kBarRowsFull + rb), (c >> 1) & 1, p.status, abort_flag);
+                const float* rows = reinterpret_cast<const float*>(smem + L.rows + rb * L.rows_bytes);
+                unsigned char* flags = smem + L.flags + rb * L.flags_bytes;
+                float* recv = reinterpret_cast<float*>(smem + L.recv + (c % kRecv) * L.recv_bytes);
+                for (int t = e; t < n; t += kEpiWarps) {
+                    const uint2 fw = *reinterpret_cast<const uint2*>(flags + t * kScanWarps);
+                    float o[CPL];
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) o[cc] = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < kScanWarps; ++w) {
+                        const uint32_t f = w < 4 ? (fw.x >> (8 * w)) & 0xFFu : (fw.y >> (8 * (w - 4))) & 0xFFu;
+                        if (f) {
+                            float pr[CPL];
+                            load_row<CPL>(reinterpret_cast<const unsigned char*>(rows), (t * kScanWarps + w) * dv + lch, 0, pr);
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) o[cc] += pr[cc];
+                        }
+                    }
+                    __syncwarp();
+                    if (lane < 2) reinterpret_cast<uint32_t*>(flags + t * kScanWarps)[lane] = 0u;
+                    // recv[r'][t][dv]: slot r' holds CTA r''s partial sums
+                    float* dst = recv + (static_cast<size_t>(rank) * C + t) * dv + lch;
+                    if (lane < LW) {
+                        if (ncta == 1) {
+                            store_row<CPL>(dst, o);
+                        } else {
+                            for (int r = 0; r < ncta; ++r) push_row<CPL>(dst, static_cast<uint32_t>(r), o);
+                        }
+                    }
                 }
-                const float inv = 1.0f / sqrtf(tot / dv + p.eps_norm);
-                if (lane_on) {
-                    const size_t th = (static_cast<size_t>(b) * p.T + t0 + t) * p.H + h;
-                    for (int k = 0; k < cpl_lane; ++k) {
-                        const int ch = ch0 + k;
-                        const int pos = t * dv + (ch % CPL) * LW + ch / CPL;
-                        const float zz = p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(zb)[t * Dr + ch - static_cast<int>(rank) * Dr])
-                                                   : reinterpret_cast<const float*>(zb)[t * Dr + ch - static_cast<int>(rank) * Dr];
-                        const float nw = p.norm_w != nullptr ? p.norm_w[ch] : 1.0f;
-                        store_out(p.y, th * dv + ch, ob[pos] * inv * nw * zz, p.out_bf16);
+                arrive_cta(bar(kBarRowsFree + rb));
+                epi_barrier();
+                if (tid == kEpiWarp0 * 32) {
+                    if (ncta == 1) {
+                        arrive_cta(bar(kBarRecv + c % kRecv));
+                    } else {
+                        for (int r = 0; r < ncta; ++r)
+                            mbar_arrive_cluster(map_to_rank(bar(kBarRecv + c % kRecv), static_cast<uint32_t>(r)));
                     }
                 }
             }
-            // every CTA has read this chunk's partial sums and every epilogue warp has
-            // written its y: clear them for chunk c + 2
-            epi_barrier();
-            float4* ob4 = reinterpret_cast<float4*>(ob);
-            for (size_t i = etid; i < L.obuf_bytes / 16; i += kEpiWarps * 32) ob4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            arrive_cta(bar(kOFree + bf));
+            // (b) chunk d = c - kLag: all CTAs' sums are in; RMSNorm, gate, y
+            if (c >= kLag) {
+                const int d = c - kLag;
+                const int n = min(C, p.T - d * C);
+                wait_bounded<true>(bar(kBarRecv + d % kRecv), (d / kRecv) & 1, p.status, abort_flag);
+                const float* recv = reinterpret_cast<const float*>(smem + L.recv + (d % kRecv) * L.recv_bytes);
+                const unsigned char* zb = stage(d) + L.z_off;
+                for (int t = e; t < n; t += kEpiWarps) {
+                    float o[CPL];
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) o[cc] = 0.0f;
+                    if (lane < LW) {
+                        for (int r = 0; r < ncta; ++r) {
+                            float pr[CPL];
+                            load_row<CPL>(reinterpret_cast<const unsigned char*>(recv), (r * C + t) * dv + lch, 0, pr);
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) o[cc] += pr[cc];
+                        }
+                    }
+                    float sq = 0.0f;
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) sq = fmaf(o[cc], o[cc], sq);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    const float inv = 1.0f / sqrtf(sq / dv + p.eps_norm);
+                    if (mine) {
+                        float zz[CPL];
+                        load_row<CPL>(zb, t * Dr + lch - static_cast<int>(rank) * Dr, p.in_bf16, zz);
+                        const size_t base = ((static_cast<size_t>(b) * p.T + d * C + t) * p.H + h) * dv + lch;
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) store_out(p.y, base + cc, o[cc] * inv * nw[cc] * zz[cc], p.out_bf16);
+                    }
+                }
+                arrive_cta(bar(kBarStageFree + d % kStages));
+            }
         }
     }
 
     // copies still in flight after an abort must land before the CTA exits
-    if (warp == kLoadWarp || warp == kEpiWarp0) {
-        const int base = warp == kLoadWarp ? kStage : kZ;
-        for (int c = max(0, nch - 2); c < nch; ++c) drain_copies(bar(base + (c & 1)), (c >> 1) & 1);
+    if (warp == kLoadWarp) {
+        for (int c = max(0, nch - kStages); c < nch; ++c) drain_copies(bar(kBarStage + c % kStages), (c / kStages) & 1);
     }
-    // no CTA leaves while a peer may still read its shared memory
+    // no CTA leaves while a peer may still write into its shared memory
     __syncthreads();
     if (ncta > 1 && tid == 0) {
-        signal_cluster(bar(kFin), ncta);
-        wait_bounded<true>(bar(kFin), 0, p.status, abort_flag);
+        for (int r = 0; r < ncta; ++r) mbar_arrive_cluster(map_to_rank(bar(kBarFin), static_cast<uint32_t>(r)));
+        wait_bounded<true>(bar(kBarFin), 0, p.status, abort_flag);
     }
     tmem_fence_before_sync();
     __syncthreads();
@@ -478,6 +544,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
 }
 
 }  // namespace
+
+size_t chunk_block_bytes(int chunk, int K, int ncta, size_t* recs_off, size_t* alph_off)
+{
+    const size_t E = static_cast<size_t>(2) * chunk * K;
+    const size_t ro = align16(sizeof(int) * (8 * ncta + 1));
+    const size_t ao = ro + align16(sizeof(uint2) * E);
+    if (recs_off) *recs_off = ro;
+    if (alph_off) *alph_off = ao;
+    return align16(ao + sizeof(float) * E);
+}
 
 bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
 {
@@ -496,16 +572,22 @@ bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
     const int cols = ((Ml + 3) / 4) * cpl;
     uint32_t alloc = 32;
     while (alloc < static_cast<uint32_t>(cols)) alloc <<= 1;
-    int C = 64;
-    while (C > 8 && (2 * C * K > 2048 || scan_layout(Ml, C, K, d_v, n, in_bytes).total > 200 * 1024)) C >>= 1;
-    const size_t total = scan_layout(Ml, C, K, d_v, n, in_bytes).total;
-    if (total > 200 * 1024) return false;
+    // output-gate columns of one CTA are copied per token with 16-byte bulk copies
+    if (d_v / n < 8) return false;
+    int C = 16;
+    auto total = [&](int cc) {
+        return scan_layout(Ml, cc, d_v, n, in_bytes, chunk_block_bytes(cc, K, n, nullptr, nullptr)).total;
+    };
+    const size_t budget = 220 * 1024;
+    while (C > 2 && total(C) > budget) C >>= 1;
+    if (total(C) > budget) return false;
     out->ncta = n;
     out->chunk = C;
     out->cpl = cpl;
     out->tmem_cols = alloc;
     // more than half of the SM's shared memory: exactly one CTA (and one TMEM owner) per SM
-    out->smem_bytes = total < 116 * 1024 ? 116 * 1024 : total;
+    const size_t t = total(C);
+    out->smem_bytes = t < 116 * 1024 ? 116 * 1024 : t;
     out->nchunks = 0;
     return true;
 }
