@@ -5,17 +5,15 @@
 // computed in parallel first, and the read/write events are grouped by slot so that
 // each slot sees its own causal sequence.  Here the grouping is by owner warp of the
 // scan kernel (a fixed set of slots per warp), keeping token order within each list:
-//   owner o = (slot mod ncta) * 8 + ((slot / ncta) mod 8)
+//   owner o = (slot mod ncta) * NW + ((slot / ncta) mod NW),  NW = scan warps per CTA
 // and, within one token, the K writes come before the K reads (the read sees the
-// token's own write).  Owners of one scan CTA are contiguous (o / 8 = CTA rank).
+// token's own write).  Owners of one scan CTA are contiguous (o / NW = CTA rank).
 //
-// Each owner list is also cut into batches of at most 8 consecutive events on distinct
-// slots; the scan kernel loads a whole batch from tensor memory with one wait.
-//
-// Output per (b, h, chunk), one contiguous block of `chunk_bytes` (see ChunkLayout):
+// Output per (b, h, chunk), one contiguous block of `chunk_bytes` (chunk_block_bytes()):
 //   offs[NO + 1]   start of each owner's segment, then the total event count
-//   recs[2*C*K]    {meta, weight}: meta = t << 16 | write << 15 | batch_len << 10 | column
-//                  (batch_len is set on the first event of each batch, 0 elsewhere)
+//   recs[2*C*K]    {meta, weight}: meta = t << 24 | j << 16 | write << 15 | column, with
+//                  t the token within the chunk, j the event's rank within its token's
+//                  read (or write) set and column the slot's first TMEM column
 //   alph[2*C*K]    GSU retention of write events (0 for reads)
 //
 // Block = (b, h, G consecutive chunks of C tokens); thread = (chunk, stream, token).  Each
@@ -57,7 +55,8 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
     const int C = p.chunk, G = p.chunks_per_block;
     const int nt = blockDim.x;         // whole warps; threads >= 2*C*G carry no token
     const int nact = 2 * C * G;        // threads: (chunk g, stream, token)
-    const int NO = 8 * p.ncta;
+    const int NW = p.nwarps;           // scan warps (owners) per CTA
+    const int NO = NW * p.ncta;
     const int E = 2 * C * p.K;         // event capacity of one chunk
     const int TS = NO * 2 * C;         // table entries of one chunk
     uint64_t* kept = reinterpret_cast<uint64_t*>(smem);                          // [KMAX][nt]
@@ -103,9 +102,9 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
                 int32_t slot = packed_index(out[j], p.M);
                 if (cape) slot = cape_shift(slot, pos, p.M);
                 const int s = slot >> lg_ncta;
-                owner[j] = (slot & (p.ncta - 1)) * 8 + (s & 7);
-                meta[j] = (static_cast<uint32_t>(tl) << 16) | (stream == 0 ? 0x8000u : 0u) |
-                          static_cast<uint32_t>((s >> 2) * p.cpl);
+                owner[j] = (slot & (p.ncta - 1)) * NW + (s & (NW - 1));
+                meta[j] = (static_cast<uint32_t>(tl) << 24) | (static_cast<uint32_t>(j) << 16) |
+                          (stream == 0 ? 0x8000u : 0u) | static_cast<uint32_t>((s >> 2) * p.cpl);
                 coef[j] = w[j];
                 alpha[j] = stream == 0 ? gsu_alpha(w[j], gg) : 0.0f;
             }
@@ -126,17 +125,13 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
     {
         const int W = (G * TS + nt - 1) / nt;
         const int lo = min(tid * W, G * TS), hi = min(lo + W, G * TS);
-        int loc[64];
         int sum = 0;
-        for (int k = 0; k < hi - lo; ++k) {
-            loc[k] = table[lo + k];
-            sum += loc[k];
-        }
-        __syncthreads();
+        for (int k = lo; k < hi; ++k) sum += table[k];
         int run = block_exclusive_scan(sum, warp_tot, &total);
-        for (int k = 0; k < hi - lo; ++k) {
-            table[lo + k] = run;
-            run += loc[k];
+        for (int k = lo; k < hi; ++k) {
+            const int v = table[k];
+            table[k] = run;
+            run += v;
         }
     }
     __syncthreads();
@@ -160,27 +155,6 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
         }
     }
     __syncthreads();
-    // batches: greedy runs of at most 8 events with distinct columns, per owner list
-    for (int i0 = tid; i0 < G * NO; i0 += nt) {
-        const int gg = i0 / NO, o = i0 - gg * NO;
-        uint2* rr = srec + gg * E;
-        int i = soff[gg * (NO + 1) + o];
-        const int end = soff[gg * (NO + 1) + o + 1];
-        while (i < end) {
-            uint32_t cols[8];
-            int nb = 0;
-            while (nb < 8 && i + nb < end) {
-                const uint32_t col = rr[i + nb].x & 0x3FFu;
-                bool dup = false;
-                for (int k = 0; k < nb; ++k) dup |= cols[k] == col;
-                if (dup) break;
-                cols[nb++] = col;
-            }
-            rr[i].x |= static_cast<uint32_t>(nb) << 10;
-            i += nb;
-        }
-    }
-    __syncthreads();
     // the chunk blocks: offsets, records, retentions
     for (int gg = 0; gg < G; ++gg) {
         const int cc = c0 + gg;
@@ -198,15 +172,14 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
     }
 }
 
+int kmax_of(int K) { return K <= 8 ? 8 : K <= 16 ? 16 : K <= 32 ? 32 : 64; }
+
 template <int KMAX, int DPMAX>
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s)
 {
     const int G = p.chunks_per_block;
     const int nt = 2 * p.chunk * G;
-    const int NO = 8 * p.ncta;
-    const int E = 2 * p.chunk * p.K;
-    const size_t smem = sizeof(uint64_t) * KMAX * ((nt + 31) / 32 * 32) + sizeof(int) * (G * NO * 2 * p.chunk + 8) +
-                        (sizeof(uint2) + sizeof(float)) * G * E + sizeof(int) * G * (NO + 1);
+    const size_t smem = route_smem_bytes(p.chunk, G, p.K, p.nwarps * p.ncta);
     auto kern = k_decode_route<KMAX, DPMAX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -227,13 +200,27 @@ cudaError_t route_k(const RouteParams& p, cudaStream_t s)
 
 }  // namespace
 
+size_t route_smem_bytes(int chunk, int G, int K, int n_owners)
+{
+    const int nt = (2 * chunk * G + 31) / 32 * 32;
+    const size_t E = static_cast<size_t>(2) * chunk * K;
+    return sizeof(uint64_t) * kmax_of(K) * nt + sizeof(int) * (static_cast<size_t>(G) * n_owners * 2 * chunk + 8) +
+           (sizeof(uint2) + sizeof(float)) * G * E + sizeof(int) * G * (n_owners + 1);
+}
+
+// as many chunks per block as fit 128 threads (a power of two)
+int route_chunks_per_block(int chunk, int nchunks)
+{
+    int G = 1;
+    while (2 * chunk * G * 2 <= 128 && G * 2 <= nchunks) G *= 2;
+    return G;
+}
+
 cudaError_t launch_decode_route(const RouteParams& p_in, cudaStream_t stream)
 {
     RouteParams p = p_in;
-    if (2 * p.chunk > 128 || 8 * p.ncta > 64) return cudaErrorInvalidValue;
-    // as many chunks per block as fit 128 threads, keeping the flattened table divisible
-    p.chunks_per_block = 1;
-    while (2 * p.chunk * p.chunks_per_block * 2 <= 128 && p.chunks_per_block * 2 <= p.nchunks) p.chunks_per_block *= 2;
+    if (2 * p.chunk > 128 || p.nwarps * p.ncta > 128) return cudaErrorInvalidValue;
+    p.chunks_per_block = route_chunks_per_block(p.chunk, p.nchunks);
     if (p.d_p <= 4) return route_k<4>(p, stream);
     if (p.d_p <= 8) return route_k<8>(p, stream);
     return route_k<16>(p, stream);

@@ -36,6 +36,7 @@ struct RouteParams {
     const int32_t* pos0;       // [B] or null
     const uint8_t* cape_mask;  // [H] or null
     int ncta, cpl, chunk, nchunks;
+    int nwarps;             // scan warps per CTA (owners per CTA)
     int chunks_per_block;   // set by the launcher
     unsigned char* blocks;  // [B*H*nchunks][chunk_bytes]
     size_t chunk_bytes, recs_off, alph_off;
@@ -63,7 +64,7 @@ struct ScanParams {
 };
 
 struct ScanPlan {
-    int ncta, chunk, cpl, nchunks;
+    int ncta, chunk, cpl, nchunks, nwarps;
     uint32_t tmem_cols;
     size_t smem_bytes;
 };
@@ -91,9 +92,12 @@ struct StepParams {
 // Returns false if the slot array does not fit.
 bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* plan);
 // Bytes of one chunk block (offsets, records, retentions) and the offsets of its parts.
-size_t chunk_block_bytes(int chunk, int K, int ncta, size_t* recs_off, size_t* alph_off);
+size_t chunk_block_bytes(int chunk, int K, int ncta, int nwarps, size_t* recs_off, size_t* alph_off);
 
 cudaError_t launch_decode_addresses(const DecodeParams& p, cudaStream_t stream);
+// Shared memory of one decode/route block of G chunks (largest G: 64 / chunk).
+size_t route_smem_bytes(int chunk, int G, int K, int n_owners);
+int route_chunks_per_block(int chunk, int nchunks);
 cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream);
 cudaError_t launch_decode_step(const StepParams& p, cudaStream_t stream);

@@ -91,7 +91,7 @@ WorkspaceLayout workspace_layout(int B, int T, int H, int K, const ramnet::ScanP
 {
     WorkspaceLayout w;
     w.nchunks = (T + plan.chunk - 1) / plan.chunk;
-    w.chunk_bytes = ramnet::chunk_block_bytes(plan.chunk, K, plan.ncta, &w.recs_off, &w.alph_off);
+    w.chunk_bytes = ramnet::chunk_block_bytes(plan.chunk, K, plan.ncta, plan.nwarps, &w.recs_off, &w.alph_off);
     w.total = static_cast<size_t>(B) * H * w.nchunks * w.chunk_bytes + 256;
     return w;
 }
@@ -128,9 +128,15 @@ size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t 
 {
     int M = 0;
     if (check_config(cfg, &M) != RAMNET_OK || check_sizes(B, T, H) != RAMNET_OK) return 0;
-    ramnet::ScanPlan plan;
-    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, 4, &plan)) return 0;
-    return workspace_layout(B, T, H, cfg->K, plan).total;
+    // the chunk length depends on the input element size: the larger of the two
+    size_t total = 0;
+    for (int in_bytes : {2, 4}) {
+        ramnet::ScanPlan plan;
+        if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_bytes, &plan)) return 0;
+        const size_t t = workspace_layout(B, T, H, cfg->K, plan).total;
+        total = t > total ? t : total;
+    }
+    return total;
 }
 
 ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
@@ -160,7 +166,7 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     OPTIONAL_PTR(S_in);
     OPTIONAL_PTR(m_in);
     ramnet::ScanPlan plan;
-    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, 4, &plan))
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, &plan))
         return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", M,
                     cfg->d_v);
     const WorkspaceLayout wl = workspace_layout(B, T, H, cfg->K, plan);
@@ -189,6 +195,7 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     rp.cpl = plan.cpl;
     rp.chunk = plan.chunk;
     rp.nchunks = wl.nchunks;
+    rp.nwarps = plan.nwarps;
     rp.blocks = static_cast<unsigned char*>(workspace);
     rp.chunk_bytes = wl.chunk_bytes;
     rp.recs_off = wl.recs_off;
