@@ -47,7 +47,8 @@
  *     a wait gives up the kernel records it in a device status word and returns early.
  *     ramnet_sync_status() reads (and clears) that word.
  *   - No call allocates device memory.  Scratch space comes from the caller
- *     (ramnet_scan_forward's workspace).
+ *     (ramnet_scan_forward's workspace) or, for ramnet_scan_forward_noalloc, from a
+ *     fixed array inside the library's device image.
  *   - Limits: 2 <= d_p <= 16, 1 <= U <= 8, M = d_p^U <= 65536, 1 <= K <= min(M, 64),
  *     d_v in {16, 32, 64, 128, 256}.  ramnet_scan_forward additionally needs the slot
  *     array of one head to fit the tensor memory of at most 8 SMs (M * max(d_v,32) *
@@ -139,6 +140,38 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
                                   const int32_t* pos0, const float* S_in, const float* m_in,
                                   void* y, ramnet_dtype out_dt, float* S_out, float* m_out,
                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Size of the scratch array built into the library for ramnet_scan_forward_noalloc. */
+#define RAMNET_NOALLOC_SCRATCH_BYTES ((size_t)32 * 1024 * 1024)
+
+/*
+ * ramnet_scan_forward_noalloc -- ramnet_scan_forward without a caller-provided workspace.
+ * The RAM-Net pages describe no such call: it exists for callers that cannot pass device
+ * memory of their own (host code without a device allocator, or a hot path on which an
+ * allocation could block or fail).  Same arguments, results and errors as
+ * ramnet_scan_forward, minus workspace and workspace_bytes.
+ *
+ *   Scratch:   a static, 256-byte aligned device array of RAMNET_NOALLOC_SCRATCH_BYTES
+ *              (32 MiB) per device, part of the library's device image.  Sizes for which
+ *              ramnet_scan_workspace_bytes() exceeds that return RAMNET_ERR_UNSUPPORTED
+ *              with a message giving both numbers.  Nothing in the array has to start at
+ *              zero: each call writes all the scratch it later reads.
+ *   Set-up:    the first call on a device (with that device current) looks up the
+ *              array's device address once and keeps it; make that first call before
+ *              beginning any stream capture.
+ *   Sharing:   all calls on a device use the same array.  Calls whose work can overlap
+ *              on the device (other streams, other host threads) race on it; issue them
+ *              on one stream, or use ramnet_scan_forward with separate workspaces.
+ *   Allocation: none, host or device.
+ */
+ramnet_status ramnet_scan_forward_noalloc(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                          ramnet_dtype in_dt, const void* k_logits,
+                                          const void* q_logits, const void* v, const void* g,
+                                          const void* z, const float* norm_w,
+                                          const uint8_t* cape_mask, const int32_t* pos0,
+                                          const float* S_in, const float* m_in, void* y,
+                                          ramnet_dtype out_dt, float* S_out, float* m_out,
+                                          void* stream);
 
 /*
  * ramnet_decode_step -- one autoregressive token per (b,h) against an HBM-resident state,

@@ -98,6 +98,17 @@ WorkspaceLayout workspace_layout(int B, int T, int H, int K, const ramnet::ScanP
 
 }  // namespace
 
+namespace ramnet {
+
+// Sets the text ramnet_last_error returns on this thread (for entry points in other files).
+ramnet_status set_last_error(ramnet_status s, const char* msg)
+{
+    g_last_error = msg;
+    return s;
+}
+
+}  // namespace ramnet
+
 extern "C" {
 
 const char* ramnet_last_error(void) { return g_last_error.c_str(); }

@@ -22,7 +22,8 @@ RAMNET_F32, RAMNET_BF16 = 0, 1
 
 # every symbol include/ramnet.h declares
 EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_forward",
-            "ramnet_decode_step", "ramnet_sync_status", "ramnet_last_error")
+            "ramnet_scan_forward_noalloc", "ramnet_decode_step", "ramnet_sync_status", "ramnet_last_error")
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # RAMNET_NOALLOC_SCRATCH_BYTES
 
 
 class RamnetError(RuntimeError):
@@ -83,6 +84,9 @@ def load() -> ctypes.CDLL:
     lib.ramnet_scan_forward.restype = ctypes.c_int
     lib.ramnet_scan_forward.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.ramnet_scan_forward_noalloc.restype = ctypes.c_int
+    lib.ramnet_scan_forward_noalloc.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                _P, _P, ctypes.c_int, _P, _P, _P]
     lib.ramnet_decode_step.restype = ctypes.c_int
     lib.ramnet_decode_step.argtypes = [C, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.c_int, _P]
@@ -171,6 +175,20 @@ def scan_forward(cfg: Config, k_logits, q_logits, v, g, z, norm_w=None, cape_mas
         ctypes.byref(c), B, T, H, _dt(k_logits), _ptr(k_logits), _ptr(q_logits), _ptr(v), _ptr(g), _ptr(z),
         _ptr(norm_w), _ptr(cape_mask), _ptr(pos0), _ptr(S_in), _ptr(m_in), _ptr(y), _dt(y), _ptr(S_out),
         _ptr(m_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y, S_out, m_out
+
+
+def scan_forward_noalloc(cfg: Config, k_logits, q_logits, v, g, z, y, S_out, m_out, norm_w=None, cape_mask=None,
+                         pos0=None, S_in=None, m_in=None, stream=None):
+    """Prefill scan on the library's built-in scratch (no workspace argument).  All outputs
+    are passed in; nothing is allocated.  Returns (y, S_out, m_out)."""
+    B, T, H, L = k_logits.shape
+    _dense(k_logits, q_logits, v, g, z, norm_w, cape_mask, pos0, S_in, m_in, y, S_out, m_out)
+    c = cfg._c()
+    _check(load().ramnet_scan_forward_noalloc(
+        ctypes.byref(c), B, T, H, _dt(k_logits), _ptr(k_logits), _ptr(q_logits), _ptr(v), _ptr(g), _ptr(z),
+        _ptr(norm_w), _ptr(cape_mask), _ptr(pos0), _ptr(S_in), _ptr(m_in), _ptr(y), _dt(y), _ptr(S_out),
+        _ptr(m_out), _stream(stream)))
     return y, S_out, m_out
 
 
