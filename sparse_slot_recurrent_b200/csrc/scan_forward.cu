@@ -85,7 +85,7 @@ __host__ __device__ inline Layout scan_layout(int Ml, int C, int K, int dv, int 
     L.z_off = L.v_off + align16(static_cast<size_t>(C) * dv * es);
     L.stage_bytes = L.z_off + align16(static_cast<size_t>(C) * dv * es);
     L.rows_bytes = align16(sizeof(float) * C * rows_per_token(K) * dv);
-    L.flags_bytes = align16(sizeof(uint64_t) * C);
+    L.flags_bytes = static_cast<size_t>(16) * C;  // one byte per read row, 16 per token
     L.recv_bytes = align16(sizeof(float) * ncta * ((C + ncta - 1) / ncta) * dv);  // [source CTA][own token][d_v]
     size_t o = 0;
     L.bars = o;
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
     float* m_s = reinterpret_cast<float*>(smem + L.m);
     float* rows = reinterpret_cast<float*>(smem + L.rows);
-    unsigned long long* flags = reinterpret_cast<unsigned long long*>(smem + L.flags);
+    unsigned char* flags = smem + L.flags;  // [C][16]: 1 where read row (t, r) was written
     auto stage = [&](int c) { return smem + L.stage + static_cast<size_t>(c % kStages) * L.stage_bytes; };
     auto recv_slot = [&](int c) { return reinterpret_cast<float*>(smem + L.recv + (c % kRecv) * L.recv_bytes); };
     const int NWc = kScanWarps;  // owners per CTA
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
         fence_mbar_init_cluster();
     }
     if (warp == 0) tmem_alloc(holder, p.tmem_cols);
-    for (int i = tid; i < C; i += kThreads) flags[i] = 0ull;
+    for (int i = tid; i < 4 * C; i += kThreads) reinterpret_cast<uint32_t*>(flags)[i] = 0u;
     for (int s = tid; s < Ml; s += kThreads)
         m_s[s] = p.m_in != nullptr ? p.m_in[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] : 0.0f;
     tmem_fence_before_sync();
@@ -381,22 +381,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             const int beg = min(max(ofs[o], 0), E);
             const int end = min(max(ofs[o + 1], beg), E);
             uint2 nxt = beg < end ? recs[beg] : make_uint2(0u, 0u);
+            float vn[CPL];  // value row of event `nxt` (writes)
+            load_row<CPL>(vb, static_cast<int>(nxt.x >> 24) * dv + lch, p.in_bf16, vn);
             int cur_t = -1, cur_r = 0;  // read row being summed
             float acc[CPL];
 #pragma unroll
             for (int cc = 0; cc < CPL; ++cc) acc[cc] = 0.0f;
             for (int i = beg; i < end; ++i) {
                 const uint2 rec = nxt;
-                if (i + 1 < end) nxt = recs[i + 1];
+                float vv[CPL];
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) vv[cc] = vn[cc];
                 const uint32_t col = rec.x & 0x3FFu;
                 const int t = static_cast<int>(rec.x >> 24);
                 const float cf = __uint_as_float(rec.y);
                 float S[CPL];
                 tmem_ld<CPL>(tq + col, S);
+                if (i + 1 < end) {
+                    nxt = recs[i + 1];
+                    load_row<CPL>(vb, static_cast<int>(nxt.x >> 24) * dv + lch, p.in_bf16, vn);
+                }
                 if (rec.x & 0x8000u) {
                     // Gated Sparse Update step 4: S += lambda * (v - S)
-                    float vv[CPL];
-                    load_row<CPL>(vb, t * dv + lch, p.in_bf16, vv);
                     tmem_wait_ld();
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) S[cc] = fmaf(cf, vv[cc] - S[cc], S[cc]);
@@ -409,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
                     if (t != cur_t || r != cur_r) {
                         if (cur_t >= 0) {
                             if (lane < LW) store_row<CPL>(rows + (cur_t * R + cur_r) * dv + lch, acc);
-                            if (lane == 0) atomicOr(&flags[cur_t], 1ull << cur_r);
+                            if (lane == 0) flags[cur_t * 16 + cur_r] = 1;
                         }
                         cur_t = t;
                         cur_r = r;
@@ -422,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             }
             if (cur_t >= 0) {
                 if (lane < LW) store_row<CPL>(rows + (cur_t * R + cur_r) * dv + lch, acc);
-                if (lane == 0) atomicOr(&flags[cur_t], 1ull << cur_r);
+                if (lane == 0) flags[cur_t * 16 + cur_r] = 1;
             }
             scan_barrier();  // every read row of the chunk is in
             // the receivers must have finished the chunk that last used this ring slot
@@ -431,7 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             // this CTA's part of each token's read: sum its rows, send it to the token's CTA
             float* slot = recv_slot(c);
             for (int t = warp; t < n; t += kScanWarps) {
-                unsigned long long fm = flags[t];
+                const uint4 fb = *reinterpret_cast<const uint4*>(flags + t * 16);
+                unsigned long long fm = 0ull;  // bit r: read row (t, r) present
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t wv = q4 == 0 ? fb.x : q4 == 1 ? fb.y : q4 == 2 ? fb.z : fb.w;
+#pragma unroll
+                    for (int by = 0; by < 4; ++by)
+                        fm |= static_cast<unsigned long long>(((wv >> (8 * by)) & 0xFFu) != 0u) << (4 * q4 + by);
+                }
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc) acc[cc] = 0.0f;
                 for (int guard = 0; fm != 0ull && guard < 64; ++guard) {
@@ -443,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
                     for (int cc = 0; cc < CPL; ++cc) acc[cc] += pr[cc];
                 }
                 __syncwarp();
-                if (lane == 0) flags[t] = 0ull;
+                if (lane == 0) *reinterpret_cast<uint4*>(flags + t * 16) = make_uint4(0u, 0u, 0u, 0u);
                 float* dst = slot + (static_cast<size_t>(rank) * Cown + t / ncta) * dv + lch;
                 const uint32_t owner = static_cast<uint32_t>(t % ncta);
                 if (lane < LW) {
