@@ -62,6 +62,16 @@ def prefill_algorithmic_bytes(w, in_bytes=2, out_bytes=2, state_in=False) -> int
     return n_th * per_th + w.B * w.H * per_head * (2 if state_in else 1)
 
 
+def recur_algorithmic_bytes(w, in_bytes=2, out_bytes=2) -> int:
+    """The recurrence launch alone: v and z in, y out per token-head, final state per head."""
+    return w.B * w.T * w.H * w.d_v * (2 * in_bytes + out_bytes) + w.B * w.H * (w.M * w.d_v * 4 + w.M * 4)
+
+
+def route_algorithmic_bytes(w, in_bytes=2) -> int:
+    """The address launch alone: key and query logits and the write gate per token-head."""
+    return w.B * w.T * w.H * (2 * w.L * in_bytes + in_bytes)
+
+
 def decode_algorithmic_bytes(w, in_bytes=2, out_bytes=2) -> int:
     """Per (b,h) per step: inputs and y, the K write rows read and written, the K read rows
     read, and the K masses read and written (fp32)."""
@@ -101,14 +111,14 @@ def kernel_source_hash() -> str:
 def recorded_traffic(kernel: str):
     """DRAM bytes per launch from a committed ncu capture, only if the kernel sources are
     unchanged since it was taken."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
-            d = json.load(f)
-        e = d[kernel]
-        if e.get("source_hash") == kernel_source_hash():
-            return e
-    except Exception:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and parts[0] == kernel and parts[1] == kernel_source_hash():
+                    return {"dram_bytes_per_launch": int(parts[2]), "source_hash": parts[1]}
+    except OSError:
         pass
     return None
 
@@ -129,7 +139,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
@@ -227,7 +237,7 @@ def oracle_sample(w, n_heads: int, threads: int):
 
 
 def cpu_baseline(w, cores: int):
-    n_heads = min(w.B * w.H, max(8, 2 * cores))
+    n_heads = w.B * w.H  # the whole workload: a few seconds on 16 cores
     secs, th = oracle_sample(w, n_heads, cores)
     heads = ((n_heads + w.H - 1) // w.H) * w.H
     return {"value": th / w.H / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -290,15 +300,22 @@ def run_gpu(args, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"], cape_mask=d["cape_mask"],
-                            pos0=d["pos0"], y=y, S_out=S, m_out=m, workspace=ws, stream=stream)
+    def route():
+        ramnet.scan_route(cfg, d["k_logits"], d["q_logits"], d["g"], ws, cape_mask=d["cape_mask"], pos0=d["pos0"],
+                          stream=stream)
 
-    launches_per_step = 3  # key decode, query decode, scan
+    def recur():
+        ramnet.scan_recur(cfg, d["v"], d["z"], y, S, m, ws, stream=stream)
+
+    def step():  # the same two launches scan_forward makes
+        route()
+        recur()
+
+    launches_per_step = 2  # decode/route, recurrence
     for _ in range(args.warmup):
         step()
     ramnet.sync_status(stream)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     clocks = ClockSampler(local)
     dist_barrier(world)
     torch.cuda.synchronize(dev)
@@ -306,27 +323,41 @@ def run_gpu(args, world, rank, local):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        step()
+        route()
         ev[i][1].record(stream)
+        recur()
+        ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
     dist_barrier(world)
     clk = clocks.stop()
     ramnet.sync_status(stream)
-    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms = statistics.mean(a.elapsed_time(c) for a, _, c in ev)
+    route_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    recur_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
     ms_max = dist_max(ms, world)
     tokens = w.B * w.T
     value = weak_scaling_value(tokens, world, ms_max)
 
-    # roofline of the timed step against measured HBM bandwidth
+    # roofline of the dominant kernel (the recurrence) against measured HBM bandwidth,
+    # plus the same figures for the address launch and the whole step
     peak, peak_kind = measured_peaks()
     nb = 2 if w.in_dtype == torch.bfloat16 else 4
+    alg_recur = recur_algorithmic_bytes(w, in_bytes=nb, out_bytes=nb)
+    alg_route = route_algorithmic_bytes(w, in_bytes=nb)
     alg = prefill_algorithmic_bytes(w, in_bytes=nb, out_bytes=nb)
-    achieved = alg / (ms / 1e3) / 1e9
-    traffic = recorded_traffic("scan_forward")
+    achieved = alg_recur / (recur_ms / 1e3) / 1e9
+    traffic = recorded_traffic("k_scan")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
-                "kernel": "ramnet_scan_forward (decode_addresses x2 + scan_tmem)",
-                "algorithmic_bytes": alg, "peak_kind": f"{peak_kind} hbm_gbs"}
+                "kernel": "k_scan (ramnet_scan_recur)", "algorithmic_bytes": alg_recur,
+                "ms_per_launch": recur_ms, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"}
+    kernels = {
+        "k_decode_route": {"ms_per_launch": route_ms, "algorithmic_bytes": alg_route,
+                           "achieved_gbs": alg_route / (route_ms / 1e3) / 1e9},
+        "k_scan": {"ms_per_launch": recur_ms, "algorithmic_bytes": alg_recur, "achieved_gbs": achieved},
+        "step": {"ms": ms, "algorithmic_bytes": alg, "achieved_gbs": alg / (ms / 1e3) / 1e9,
+                 "frac": alg / (ms / 1e3) / 1e9 / peak},
+    }
 
     # end to end through the public API from pinned host memory
     e2e = None
@@ -365,7 +396,7 @@ def run_gpu(args, world, rank, local):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; shapes of the 340M-like layer)",
-                "config": config_of(w, world), "roofline": roofline, "e2e": e2e,
+                "config": config_of(w, world), "roofline": roofline, "kernels": kernels, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk, "decode": decode}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, os.cpu_count() or 1)
@@ -434,7 +465,7 @@ def run_decode(args, world, local):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ramnet", "reference"], default="ramnet")
     ap.add_argument("--workload", default=PREFILL, choices=[k for k, v in WORKLOADS.items() if not v.decode],

@@ -141,6 +141,34 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
                                   void* y, ramnet_dtype out_dt, float* S_out, float* m_out,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ramnet_scan_route, ramnet_scan_recur -- ramnet_scan_forward in its two launches, for
+ * callers that time or schedule them apart.  ramnet_scan_forward(...) is exactly
+ * ramnet_scan_route(...) followed on the same stream by ramnet_scan_recur(...) with the
+ * same cfg, B, T, H, in_dt and workspace.
+ *
+ * ramnet_scan_route: the address decoder for every token and stream (Product-Softmax
+ *   Top-K, weights, CAPE; project page, Product Softmax and CAPE paragraphs), the write
+ *   retentions of GSU step 1, and the grouping of all read and write events by the scan
+ *   warp that owns their slot (GPU-execution paragraph: addresses for all tokens first,
+ *   events grouped by slot).  Reads k_logits, q_logits, g, cape_mask, pos0 as in
+ *   ramnet_scan_forward; writes the workspace (contents on entry ignored).
+ * ramnet_scan_recur: the recurrence (GSU steps 1-4, sparse read after the token's write,
+ *   RMSNorm, norm weight, output gate) over the events in the workspace, which must hold
+ *   what ramnet_scan_route wrote for the same arguments; the workspace is only read.
+ *   v, z, norm_w, S_in, m_in, y, S_out, m_out as in ramnet_scan_forward.
+ * Errors: as ramnet_scan_forward.
+ */
+ramnet_status ramnet_scan_route(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                ramnet_dtype in_dt, const void* k_logits, const void* q_logits,
+                                const void* g, const uint8_t* cape_mask, const int32_t* pos0,
+                                void* workspace, size_t workspace_bytes, void* stream);
+ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                ramnet_dtype in_dt, const void* v, const void* z,
+                                const float* norm_w, const float* S_in, const float* m_in, void* y,
+                                ramnet_dtype out_dt, float* S_out, float* m_out,
+                                const void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the scratch array built into the library for ramnet_scan_forward_noalloc. */
 #define RAMNET_NOALLOC_SCRATCH_BYTES ((size_t)32 * 1024 * 1024)
 

@@ -150,43 +150,35 @@ size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t 
     return total;
 }
 
-ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
-                                  const void* k_logits, const void* q_logits, const void* v, const void* g,
-                                  const void* z, const float* norm_w, const uint8_t* cape_mask, const int32_t* pos0,
-                                  const float* S_in, const float* m_in, void* y, ramnet_dtype out_dt, float* S_out,
-                                  float* m_out, void* workspace, size_t workspace_bytes, void* stream)
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the three prefill entry points; on success fills M, the plan and the
+// workspace layout.
+ramnet_status check_scan(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                         const void* workspace, size_t workspace_bytes, int* M, ramnet::ScanPlan* plan,
+                         WorkspaceLayout* wl)
 {
-    g_last_error.clear();
-    int M = 0;
-    ramnet_status st = check_config(cfg, &M);
+    ramnet_status st = check_config(cfg, M);
     if (st != RAMNET_OK) return st;
     if ((st = check_sizes(B, T, H)) != RAMNET_OK) return st;
-    if (!valid_dtype(in_dt) || !valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
-    REQUIRE_PTR(k_logits);
-    REQUIRE_PTR(q_logits);
-    REQUIRE_PTR(v);
-    REQUIRE_PTR(g);
-    REQUIRE_PTR(z);
-    REQUIRE_PTR(y);
-    REQUIRE_PTR(S_out);
-    REQUIRE_PTR(m_out);
+    if (!valid_dtype(in_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
     REQUIRE_PTR(workspace);
-    OPTIONAL_PTR(norm_w);
-    OPTIONAL_PTR(cape_mask);
-    OPTIONAL_PTR(pos0);
-    OPTIONAL_PTR(S_in);
-    OPTIONAL_PTR(m_in);
-    ramnet::ScanPlan plan;
-    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, &plan))
-        return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", M,
+    if (!ramnet::scan_plan(*M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, plan))
+        return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", *M,
                     cfg->d_v);
-    const WorkspaceLayout wl = workspace_layout(B, T, H, cfg->K, plan);
-    if (workspace_bytes < wl.total)
-        return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, wl.total);
-    uint32_t* status = device_status_ptr();
-    if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    *wl = workspace_layout(B, T, H, cfg->K, *plan);
+    if (workspace_bytes < wl->total)
+        return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, wl->total);
+    return RAMNET_OK;
+}
 
+ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt, int M,
+                         const ramnet::ScanPlan& plan, const WorkspaceLayout& wl, const void* k_logits,
+                         const void* q_logits, const void* g, const uint8_t* cape_mask, const int32_t* pos0,
+                         void* workspace, cudaStream_t s)
+{
     ramnet::RouteParams rp{};
     rp.k_logits = k_logits;
     rp.q_logits = q_logits;
@@ -213,9 +205,18 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     rp.alph_off = wl.alph_off;
     cudaError_t e = ramnet::launch_decode_route(rp, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan: decode/route launch");
+    return RAMNET_OK;
+}
 
+ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt, int M,
+                         const ramnet::ScanPlan& plan, const WorkspaceLayout& wl, const void* v, const void* z,
+                         const float* norm_w, const float* S_in, const float* m_in, void* y, ramnet_dtype out_dt,
+                         float* S_out, float* m_out, void* workspace, cudaStream_t s)
+{
+    uint32_t* status = device_status_ptr();
+    if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
     ramnet::ScanParams sp{};
-    sp.blocks = rp.blocks;
+    sp.blocks = static_cast<unsigned char*>(workspace);
     sp.chunk_bytes = wl.chunk_bytes;
     sp.recs_off = wl.recs_off;
     sp.alph_off = wl.alph_off;
@@ -241,9 +242,89 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     sp.eps_norm = cfg->eps_norm;
     sp.tmem_cols = plan.tmem_cols;
     sp.status = status;
-    e = ramnet::launch_scan(sp, plan.smem_bytes, s);
+    cudaError_t e = ramnet::launch_scan(sp, plan.smem_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return RAMNET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                                  const void* k_logits, const void* q_logits, const void* v, const void* g,
+                                  const void* z, const float* norm_w, const uint8_t* cape_mask, const int32_t* pos0,
+                                  const float* S_in, const float* m_in, void* y, ramnet_dtype out_dt, float* S_out,
+                                  float* m_out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet::ScanPlan plan;
+    WorkspaceLayout wl;
+    ramnet_status st = check_scan(cfg, B, T, H, in_dt, workspace, workspace_bytes, &M, &plan, &wl);
+    if (st != RAMNET_OK) return st;
+    if (!valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
+    REQUIRE_PTR(k_logits);
+    REQUIRE_PTR(q_logits);
+    REQUIRE_PTR(v);
+    REQUIRE_PTR(g);
+    REQUIRE_PTR(z);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(S_out);
+    REQUIRE_PTR(m_out);
+    OPTIONAL_PTR(norm_w);
+    OPTIONAL_PTR(cape_mask);
+    OPTIONAL_PTR(pos0);
+    OPTIONAL_PTR(S_in);
+    OPTIONAL_PTR(m_in);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = route_part(cfg, B, T, H, in_dt, M, plan, wl, k_logits, q_logits, g, cape_mask, pos0, workspace, s);
+    if (st != RAMNET_OK) return st;
+    return recur_part(cfg, B, T, H, in_dt, M, plan, wl, v, z, norm_w, S_in, m_in, y, out_dt, S_out, m_out, workspace,
+                      s);
+}
+
+ramnet_status ramnet_scan_route(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                                const void* k_logits, const void* q_logits, const void* g, const uint8_t* cape_mask,
+                                const int32_t* pos0, void* workspace, size_t workspace_bytes, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet::ScanPlan plan;
+    WorkspaceLayout wl;
+    ramnet_status st = check_scan(cfg, B, T, H, in_dt, workspace, workspace_bytes, &M, &plan, &wl);
+    if (st != RAMNET_OK) return st;
+    REQUIRE_PTR(k_logits);
+    REQUIRE_PTR(q_logits);
+    REQUIRE_PTR(g);
+    OPTIONAL_PTR(cape_mask);
+    OPTIONAL_PTR(pos0);
+    return route_part(cfg, B, T, H, in_dt, M, plan, wl, k_logits, q_logits, g, cape_mask, pos0, workspace,
+                      static_cast<cudaStream_t>(stream));
+}
+
+ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                                const void* v, const void* z, const float* norm_w, const float* S_in,
+                                const float* m_in, void* y, ramnet_dtype out_dt, float* S_out, float* m_out,
+                                const void* workspace, size_t workspace_bytes, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet::ScanPlan plan;
+    WorkspaceLayout wl;
+    ramnet_status st = check_scan(cfg, B, T, H, in_dt, workspace, workspace_bytes, &M, &plan, &wl);
+    if (st != RAMNET_OK) return st;
+    if (!valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
+    REQUIRE_PTR(v);
+    REQUIRE_PTR(z);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(S_out);
+    REQUIRE_PTR(m_out);
+    OPTIONAL_PTR(norm_w);
+    OPTIONAL_PTR(S_in);
+    OPTIONAL_PTR(m_in);
+    return recur_part(cfg, B, T, H, in_dt, M, plan, wl, v, z, norm_w, S_in, m_in, y, out_dt, S_out, m_out,
+                      const_cast<void*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H, ramnet_dtype in_dt,

@@ -22,7 +22,8 @@ RAMNET_F32, RAMNET_BF16 = 0, 1
 
 # every symbol include/ramnet.h declares
 EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_forward",
-            "ramnet_scan_forward_noalloc", "ramnet_decode_step", "ramnet_sync_status", "ramnet_last_error")
+            "ramnet_scan_route", "ramnet_scan_recur", "ramnet_scan_forward_noalloc", "ramnet_decode_step",
+            "ramnet_sync_status", "ramnet_last_error")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # RAMNET_NOALLOC_SCRATCH_BYTES
 
 
@@ -84,6 +85,11 @@ def load() -> ctypes.CDLL:
     lib.ramnet_scan_forward.restype = ctypes.c_int
     lib.ramnet_scan_forward.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.ramnet_scan_route.restype = ctypes.c_int
+    lib.ramnet_scan_route.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.ramnet_scan_recur.restype = ctypes.c_int
+    lib.ramnet_scan_recur.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P,
+                                      _P, ctypes.c_size_t, _P]
     lib.ramnet_scan_forward_noalloc.restype = ctypes.c_int
     lib.ramnet_scan_forward_noalloc.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                 _P, _P, ctypes.c_int, _P, _P, _P]
@@ -175,6 +181,28 @@ def scan_forward(cfg: Config, k_logits, q_logits, v, g, z, norm_w=None, cape_mas
         ctypes.byref(c), B, T, H, _dt(k_logits), _ptr(k_logits), _ptr(q_logits), _ptr(v), _ptr(g), _ptr(z),
         _ptr(norm_w), _ptr(cape_mask), _ptr(pos0), _ptr(S_in), _ptr(m_in), _ptr(y), _dt(y), _ptr(S_out),
         _ptr(m_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y, S_out, m_out
+
+
+def scan_route(cfg: Config, k_logits, q_logits, g, workspace, cape_mask=None, pos0=None, stream=None):
+    """First launch of scan_forward: address decode, CAPE, write retentions, event grouping
+    into ``workspace`` (uint8 device tensor of at least scan_workspace_bytes())."""
+    B, T, H, L = k_logits.shape
+    _dense(k_logits, q_logits, g, cape_mask, pos0, workspace)
+    c = cfg._c()
+    _check(load().ramnet_scan_route(ctypes.byref(c), B, T, H, _dt(k_logits), _ptr(k_logits), _ptr(q_logits), _ptr(g),
+                                    _ptr(cape_mask), _ptr(pos0), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def scan_recur(cfg: Config, v, z, y, S_out, m_out, workspace, norm_w=None, S_in=None, m_in=None, stream=None):
+    """Second launch of scan_forward: the recurrence over the events scan_route wrote."""
+    B, T, H, dv = v.shape
+    _dense(v, z, y, S_out, m_out, workspace, norm_w, S_in, m_in)
+    c = cfg._c()
+    _check(load().ramnet_scan_recur(ctypes.byref(c), B, T, H, _dt(v), _ptr(v), _ptr(z), _ptr(norm_w), _ptr(S_in),
+                                    _ptr(m_in), _ptr(y), _dt(y), _ptr(S_out), _ptr(m_out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
     return y, S_out, m_out
 
 

@@ -190,6 +190,28 @@ def test_scan_matches_oracle(case):
     assert _maxabs(m, om) <= tol
 
 
+def test_scan_route_then_recur_matches_oracle_and_forward():
+    """The two-launch form (route, then recurrence over the workspace) gives the oracle's
+    results and exactly the single-call results."""
+    w, inp = _small_inputs(4, 4, 16, 64, 2, 233, 2, torch.bfloat16, "normal", seed=21)
+    cfg, ocfg = _cfgs(w)
+    g = torch.Generator().manual_seed(22)
+    S_in = torch.randn((2, 2, w.M, 64), generator=g)
+    m_in = torch.rand((2, 2, w.M), generator=g) * 2
+    y0, S0, m0 = _gpu_scan(cfg, inp, None, S_in, m_in)
+    d = _cuda(inp)
+    ws = torch.empty(ramnet.scan_workspace_bytes(cfg, 2, 233, 2), dtype=torch.uint8, device="cuda")
+    y = torch.empty((2, 233, 2, 64), dtype=torch.float32, device="cuda")
+    S = torch.empty((2, 2, w.M, 64), dtype=torch.float32, device="cuda")
+    m = torch.empty((2, 2, w.M), dtype=torch.float32, device="cuda")
+    ramnet.scan_route(cfg, d["k_logits"], d["q_logits"], d["g"], ws, cape_mask=d["cape_mask"], pos0=d["pos0"])
+    ramnet.scan_recur(cfg, d["v"], d["z"], y, S, m, ws, S_in=S_in.cuda(), m_in=m_in.cuda())
+    ramnet.sync_status()
+    oy, oS, om = _oracle_scan(ocfg, inp, None, S_in, m_in)
+    assert _maxabs(y, oy) <= TOL_BF16 and _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
+    assert torch.equal(y.cpu(), y0.cpu()) and torch.equal(S.cpu(), S0.cpu()) and torch.equal(m.cpu(), m0.cpu())
+
+
 def test_scan_unselected_slots_bit_identical():
     """Rows and masses of slots no token writes come back exactly as they went in."""
     w, inp = _small_inputs(4, 5, 8, 128, 2, 96, 2, torch.bfloat16, "mixed", seed=3)
