@@ -220,6 +220,18 @@ ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H,
                                  void* y, ramnet_dtype out_dt, void* stream);
 
 /*
+ * ramnet_selftest_wait_timeout -- failure-detection self-test.  The pages have no
+ * counterpart: it checks this library's own guard against lost signals.  Launches one
+ * block on `stream` whose bounded wait (the same routine every wait of the prefill scan
+ * uses) is on a barrier that nothing signals, so it gives up after limit_us microseconds
+ * and records RAMNET_ERR_TIMEOUT in the device status word; the next
+ * ramnet_sync_status(stream) returns RAMNET_ERR_TIMEOUT and clears it.  No fault, trap
+ * or hang is involved and the context stays usable.
+ * Errors: INVALID_ARG unless 1 <= limit_us <= 2000000.
+ */
+ramnet_status ramnet_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/*
  * ramnet_sync_status -- waits for `stream`, then returns RAMNET_ERR_TIMEOUT or
  * RAMNET_ERR_DEVICE_CHECK if a kernel of this library on the current device recorded a
  * gave-up wait or a failed check since the last call (and clears the record), or

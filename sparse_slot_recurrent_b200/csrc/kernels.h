@@ -100,6 +100,8 @@ size_t route_smem_bytes(int chunk, int G, int K, int n_owners);
 int route_chunks_per_block(int chunk, int nchunks);
 cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream);
+// One block whose bounded wait on a never-signalled barrier runs out after limit_ns.
+cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_decode_step(const StepParams& p, cudaStream_t stream);
 
 }  // namespace ramnet

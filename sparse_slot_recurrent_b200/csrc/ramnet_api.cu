@@ -327,6 +327,18 @@ ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, 
                       const_cast<void*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
+ramnet_status ramnet_selftest_wait_timeout(uint32_t limit_us, void* stream)
+{
+    g_last_error.clear();
+    if (limit_us < 1 || limit_us > 2000000) return fail(RAMNET_ERR_INVALID_ARG, "limit_us=%u outside [1, 2000000]", limit_us);
+    uint32_t* status = device_status_ptr();
+    if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+    cudaError_t e = ramnet::launch_wait_selftest(status, static_cast<uint64_t>(limit_us) * 1000ull,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+    return RAMNET_OK;
+}
+
 ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H, ramnet_dtype in_dt,
                                  const void* k_logits, const void* q_logits, const void* v, const void* g,
                                  const void* z, const float* norm_w, const uint8_t* cape_mask, const int32_t* pos,

@@ -144,14 +144,15 @@ __device__ __forceinline__ bool try_wait_clu(uint32_t bar, uint32_t parity)
 }
 
 // Bounded wait for phase `parity` of the mbarrier at shared address `bar`: at most
-// kSpinLimit polls and about 2 s.  On expiry the status word gets kDevTimeout and the
-// CTA's abort flag is raised, after which every later wait of the CTA returns at once,
-// so a kernel that lost a signal still ends within a few seconds.
+// kSpinLimit polls and `limit_ns` (2 s unless given).  On expiry the status word gets
+// kDevTimeout and the CTA's abort flag is raised, after which every later wait of the CTA
+// returns at once, so a kernel that lost a signal still ends within a few seconds.
 template <bool kCluster>
-__device__ __noinline__ void wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag)
+__device__ __noinline__ void wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag,
+                                          uint64_t limit_ns = 2000000000ull)
 {
     if (*abort_flag) return;
-    const uint64_t t_end = global_ns() + 2000000000ull;
+    const uint64_t t_end = global_ns() + limit_ns;
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
         if (kCluster ? try_wait_clu(bar, parity) : try_wait_cta(bar, parity)) return;
         if (global_ns() > t_end || *abort_flag) break;
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const int C = p.chunk, dv = p.d_v, ncta = p.ncta, M = p.M, K = p.K;
-    const int LW = dv < 32 ? dv : 32;  // lanes holding channels
+    const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;  // lanes holding channels (32 unless d_v = 16)
     const int es = p.in_bf16 ? 2 : 4;
     const uint32_t rank = ncta > 1 ? cluster_ctarank() : 0u;
     const int bh = blockIdx.x / ncta;
@@ -408,17 +409,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
                     for (int cc = 0; cc < CPL; ++cc) S[cc] = fmaf(cf, vv[cc] - S[cc], S[cc]);
                     tmem_st<CPL>(tq + col, S);
                     tmem_wait_st();
-                } else {
-                    // read: weighted row, summed into read row (t, r)
-                    const int r = byw ? warp : static_cast<int>((rec.x >> 16) & 0x3Fu);
+                } else if (!byw) {
+                    // read j of token t: its weighted row goes straight to read row (t, j)
+                    const int j = static_cast<int>((rec.x >> 16) & 0x3Fu);
                     tmem_wait_ld();
-                    if (t != cur_t || r != cur_r) {
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) S[cc] *= cf;
+                    if (lane < LW) store_row<CPL>(rows + (t * R + j) * dv + lch, S);
+                    flags[t * 16 + j] = 1;  // every lane stores the same byte
+                } else {
+                    // read, K > kScanWarps: summed into read row (t, warp) first
+                    tmem_wait_ld();
+                    if (t != cur_t) {
                         if (cur_t >= 0) {
                             if (lane < LW) store_row<CPL>(rows + (cur_t * R + cur_r) * dv + lch, acc);
-                            if (lane == 0) flags[cur_t * 16 + cur_r] = 1;
+                            flags[cur_t * 16 + cur_r] = 1;
                         }
                         cur_t = t;
-                        cur_r = r;
+                        cur_r = warp;
 #pragma unroll
                         for (int cc = 0; cc < CPL; ++cc) acc[cc] = 0.0f;
                     }
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             }
             if (cur_t >= 0) {
                 if (lane < LW) store_row<CPL>(rows + (cur_t * R + cur_r) * dv + lch, acc);
-                if (lane == 0) flags[cur_t * 16 + cur_r] = 1;
+                flags[cur_t * 16 + cur_r] = 1;
             }
             scan_barrier();  // every read row of the chunk is in
             // the receivers must have finished the chunk that last used this ring slot
@@ -617,7 +625,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
     if (warp == 0) tmem_dealloc(tbase, p.tmem_cols);
 }
 
+// Failure-detection self-test: one thread waits, through wait_bounded, on a barrier that
+// nothing ever signals; the wait gives up after limit_ns and records kDevTimeout.
+__global__ void k_wait_selftest(uint32_t* status, uint64_t limit_ns)
+{
+    __shared__ uint64_t never;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&never, 1);
+        fence_mbar_init_cluster();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) wait_bounded<false>(smem_addr(&never), 0, status, &abort_flag, limit_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream)
+{
+    k_wait_selftest<<<1, 32, 0, stream>>>(status, limit_ns);
+    return cudaGetLastError();
+}
 
 size_t chunk_block_bytes(int chunk, int K, int ncta, int nwarps, size_t* recs_off, size_t* alph_off)
 {

@@ -23,7 +23,7 @@ RAMNET_F32, RAMNET_BF16 = 0, 1
 # every symbol include/ramnet.h declares
 EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_forward",
             "ramnet_scan_route", "ramnet_scan_recur", "ramnet_scan_forward_noalloc", "ramnet_decode_step",
-            "ramnet_sync_status", "ramnet_last_error")
+            "ramnet_selftest_wait_timeout", "ramnet_sync_status", "ramnet_last_error")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # RAMNET_NOALLOC_SCRATCH_BYTES
 
 
@@ -96,6 +96,8 @@ def load() -> ctypes.CDLL:
     lib.ramnet_decode_step.restype = ctypes.c_int
     lib.ramnet_decode_step.argtypes = [C, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.c_int, _P]
+    lib.ramnet_selftest_wait_timeout.restype = ctypes.c_int
+    lib.ramnet_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
     lib.ramnet_sync_status.restype = ctypes.c_int
     lib.ramnet_sync_status.argtypes = [_P]
     lib.ramnet_last_error.restype = ctypes.c_char_p
@@ -233,6 +235,11 @@ def decode_step(cfg: Config, k_logits, q_logits, v, g, z, S, m, pos=None, norm_w
                                      _ptr(g), _ptr(z), _ptr(norm_w), _ptr(cape_mask), _ptr(pos), _ptr(S), _ptr(m),
                                      _ptr(y), _dt(y), _stream(stream)))
     return y
+
+
+def selftest_wait_timeout(limit_us: int, stream=None):
+    """Launch the failure-detection self-test (a bounded wait that must run out)."""
+    _check(load().ramnet_selftest_wait_timeout(limit_us, _stream(stream)))
 
 
 def sync_status(stream=None):
