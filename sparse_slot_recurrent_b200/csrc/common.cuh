@@ -23,6 +23,42 @@ __device__ __forceinline__ float load_in(const void* p, size_t i, int is_bf16)
     return reinterpret_cast<const float*>(p)[i];
 }
 
+// N consecutive fp32 values from / to global memory, vectorised (p aligned to 4*N bytes,
+// or 16 bytes for N = 8).
+template <int N>
+__device__ __forceinline__ void load_row_g(const float* p, float (&v)[N])
+{
+    if constexpr (N == 1) {
+        v[0] = p[0];
+    } else if constexpr (N == 2) {
+        const float2 a = *reinterpret_cast<const float2*>(p);
+        v[0] = a.x;
+        v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(p + i);
+            v[i] = a.x;
+            v[i + 1] = a.y;
+            v[i + 2] = a.z;
+            v[i + 3] = a.w;
+        }
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void store_row_g(float* p, const float (&v)[N])
+{
+    if constexpr (N == 1) {
+        p[0] = v[0];
+    } else if constexpr (N == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) *reinterpret_cast<float4*>(p + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    }
+}
+
 __device__ __forceinline__ void store_out(void* p, size_t i, float x, int is_bf16)
 {
     if (is_bf16) reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
