@@ -50,7 +50,10 @@ __global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
             const void* lg = stream == 0 ? p.k_logits : p.q_logits;
             const size_t off = static_cast<size_t>(bh) * L;
             uint64_t out[KMAX];
-            topk_search<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, &kept_s[0][lane], 32, out);
+            if constexpr (KMAX <= 16)
+                topk_search_net<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, out);  // kept list in registers
+            else
+                topk_search<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, &kept_s[0][lane], 32, out);
             float w[KMAX];
             topk_weights<KMAX>(out, K, p.renorm, lg, off, p.in_bf16, p.d_p, p.U, w);
             const int h = bh % p.H, b = bh / p.H;

@@ -116,6 +116,81 @@ __device__ __forceinline__ void topk_search(const void* logits, size_t off, int 
     }
 }
 
+// Compare-exchange keeping the larger word in a.
+__host__ __device__ __forceinline__ void cx_desc(uint64_t& a, uint64_t& b)
+{
+    const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+    a = hi;
+    b = lo;
+}
+
+// The N largest of two descending lists of N, descending, into a: the element-wise
+// maximum of a and reversed b is a bitonic sequence holding the N largest, and a bitonic
+// merge sorts it.
+template <int N>
+__host__ __device__ __forceinline__ void merge_top(uint64_t (&a)[N], const uint64_t (&b)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; ++i) a[i] = a[i] > b[N - 1 - i] ? a[i] : b[N - 1 - i];
+#pragma unroll
+    for (int d = N / 2; d > 0; d >>= 1)
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            if ((i & d) == 0) cx_desc(a[i], a[i + d]);
+}
+
+// One level of the search with the kept list in registers (N = 8 or 16 >= K).  Digit j's
+// candidates f_i + e_j (f_i the extended kept prefix i < nk, descending in i) form a
+// descending list; invalid entries are 0, below every real candidate (a real word is at
+// least 2^48).  The lists are merged one after another into the N best, descending.
+template <int N, int DPMAX>
+__host__ __device__ __forceinline__ void topk_level_net(uint64_t (&kept)[N], int nk, const uint64_t (&e)[DPMAX], int d_p)
+{
+    const uint64_t mul = static_cast<uint64_t>(d_p - 1);
+    uint64_t f[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) f[i] = kept[i] + (kept[i] & 0xFFFFull) * mul;
+    uint64_t acc[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) acc[i] = i < nk ? f[i] + e[0] : 0ull;
+#pragma unroll
+    for (int j = 1; j < DPMAX; ++j) {
+        if (j < d_p) {
+            uint64_t l[N];
+#pragma unroll
+            for (int i = 0; i < N; ++i) l[i] = i < nk ? f[i] + e[j] : 0ull;
+            merge_top<N>(acc, l);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) kept[i] = acc[i];
+}
+
+// Exact Top-K (K <= N) with the kept list in registers: the same result as topk_search,
+// since the candidate words are distinct and the N best are therefore unique.
+template <int N, int DPMAX>
+__device__ __forceinline__ void topk_search_net(const void* logits, size_t off, int is_bf16, int d_p, int U, int K,
+                                                uint64_t (&out)[N])
+{
+    uint64_t kept[N];
+    kept[0] = kKeyBias << 16;  // the empty prefix: score 0, low 0
+#pragma unroll
+    for (int i = 1; i < N; ++i) kept[i] = 0ull;
+    int nk = 1;
+    for (int u = 0; u < U; ++u) {
+        uint64_t e[DPMAX];
+#pragma unroll
+        for (int d = 0; d < DPMAX; ++d) e[d] = d < d_p ? digit_code(load_in(logits, off + u * d_p + d, is_bf16), d, d_p) : 0ull;
+        topk_level_net<N, DPMAX>(kept, nk, e, d_p);
+        nk = min(K, nk * d_p);
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            if (i >= nk) kept[i] = 0ull;  // only the K best prefixes are kept
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = kept[i];
+}
+
 // Winner j's slot index (before CAPE) and score.
 __device__ __forceinline__ int32_t packed_index(uint64_t p, int32_t M) { return (M - 1) - static_cast<int32_t>(p & 0xFFFFull); }
 __device__ __forceinline__ int64_t packed_score(uint64_t p) { return static_cast<int64_t>((p >> 16) - kKeyBias); }
