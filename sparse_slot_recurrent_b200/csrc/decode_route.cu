@@ -95,6 +95,11 @@ __global__ void __launch_bounds__(128) k_decode_route(RouteParams p)
         const bool cape = p.cape_mask != nullptr && p.cape_mask[h] != 0;
         const int64_t pos = static_cast<int64_t>(p.pos0 != nullptr ? p.pos0[b] : 0) + t;
         const float gg = stream == 0 ? load_in(p.g, th, p.in_bf16) : 0.0f;
+        if (stream == 0) {
+            // the read accumulator of this token-head starts at zero
+            float4* orow = reinterpret_cast<float4*>(p.o + th * p.d_v);
+            for (int i = 0; i < p.d_v / 4; ++i) orow[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
         const int lg_ncta = __ffs(p.ncta) - 1;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {

@@ -40,6 +40,8 @@ struct RouteParams {
     int chunks_per_block;   // set by the launcher
     unsigned char* blocks;  // [B*H*nchunks][chunk_bytes]
     size_t chunk_bytes, recs_off, alph_off;
+    float* o;               // [B,T,H,d_v] read accumulator, zeroed here
+    int d_v;
 };
 
 struct ScanParams {
@@ -61,6 +63,7 @@ struct ScanParams {
     float eps_gsu, eps_norm;
     uint32_t tmem_cols;
     uint32_t* status;
+    float* o;  // [B,T,H,d_v] read accumulator (zeroed by the route kernel)
 };
 
 struct ScanPlan {

@@ -81,18 +81,21 @@ uint32_t* device_status_ptr()
 }
 
 // Scratch of the prefill scan: one block per (b, h, chunk) with the owner offsets, the
-// owner-sorted event records and the write retentions, plus padding for bulk copies.
+// owner-sorted event records and the write retentions, then the fp32 read accumulator
+// [B,T,H,d_v] at a 256-byte boundary.
 struct WorkspaceLayout {
-    size_t chunk_bytes, recs_off, alph_off, total;
+    size_t chunk_bytes, recs_off, alph_off, o_off, total;
     int nchunks;
 };
 
-WorkspaceLayout workspace_layout(int B, int T, int H, int K, const ramnet::ScanPlan& plan)
+WorkspaceLayout workspace_layout(int B, int T, int H, int K, int d_v, const ramnet::ScanPlan& plan)
 {
     WorkspaceLayout w;
     w.nchunks = (T + plan.chunk - 1) / plan.chunk;
     w.chunk_bytes = ramnet::chunk_block_bytes(plan.chunk, K, plan.ncta, plan.nwarps, &w.recs_off, &w.alph_off);
-    w.total = static_cast<size_t>(B) * H * w.nchunks * w.chunk_bytes + 256;
+    const size_t blocks = static_cast<size_t>(B) * H * w.nchunks * w.chunk_bytes;
+    w.o_off = (blocks + 255) & ~static_cast<size_t>(255);
+    w.total = w.o_off + static_cast<size_t>(B) * T * H * d_v * sizeof(float);
     return w;
 }
 
@@ -144,7 +147,7 @@ size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t 
     for (int in_bytes : {2, 4}) {
         ramnet::ScanPlan plan;
         if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_bytes, &plan)) return 0;
-        const size_t t = workspace_layout(B, T, H, cfg->K, plan).total;
+        const size_t t = workspace_layout(B, T, H, cfg->K, cfg->d_v, plan).total;
         total = t > total ? t : total;
     }
     return total;
@@ -168,7 +171,7 @@ ramnet_status check_scan(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     if (!ramnet::scan_plan(*M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, plan))
         return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", *M,
                     cfg->d_v);
-    *wl = workspace_layout(B, T, H, cfg->K, *plan);
+    *wl = workspace_layout(B, T, H, cfg->K, cfg->d_v, *plan);
     if (workspace_bytes < wl->total)
         return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, wl->total);
     return RAMNET_OK;
@@ -203,6 +206,8 @@ ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     rp.chunk_bytes = wl.chunk_bytes;
     rp.recs_off = wl.recs_off;
     rp.alph_off = wl.alph_off;
+    rp.o = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + wl.o_off);
+    rp.d_v = cfg->d_v;
     cudaError_t e = ramnet::launch_decode_route(rp, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan: decode/route launch");
     return RAMNET_OK;
@@ -242,6 +247,7 @@ ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     sp.eps_norm = cfg->eps_norm;
     sp.tmem_cols = plan.tmem_cols;
     sp.status = status;
+    sp.o = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + wl.o_off);
     cudaError_t e = ramnet::launch_scan(sp, plan.smem_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return RAMNET_OK;

@@ -192,7 +192,7 @@ def test_scan_matches_oracle(case):
 
 def test_scan_route_then_recur_matches_oracle_and_forward():
     """The two-launch form (route, then recurrence over the workspace) gives the oracle's
-    results and exactly the single-call results."""
+    results and the single-call results (the state exactly)."""
     w, inp = _small_inputs(4, 4, 16, 64, 2, 233, 2, torch.bfloat16, "normal", seed=21)
     cfg, ocfg = _cfgs(w)
     g = torch.Generator().manual_seed(22)
@@ -209,7 +209,10 @@ def test_scan_route_then_recur_matches_oracle_and_forward():
     ramnet.sync_status()
     oy, oS, om = _oracle_scan(ocfg, inp, None, S_in, m_in)
     assert _maxabs(y, oy) <= TOL_BF16 and _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
-    assert torch.equal(y.cpu(), y0.cpu()) and torch.equal(S.cpu(), S0.cpu()) and torch.equal(m.cpu(), m0.cpu())
+    # the state is computed in a fixed order and comes out identical; y adds its K read rows
+    # in whatever order they arrive, so it agrees to rounding
+    assert torch.equal(S.cpu(), S0.cpu()) and torch.equal(m.cpu(), m0.cpu())
+    assert _maxabs(y, y0) <= TOL_F32
 
 
 def test_scan_unselected_slots_bit_identical():
