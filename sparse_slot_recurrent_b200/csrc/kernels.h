@@ -21,11 +21,8 @@ struct DecodeParams {
     float* w_out;              // [B,T,H,K]
 };
 
-// Decode + route (first kernel of the prefill scan): per (b, h, chunk) the token-ordered
-// event list of every owner warp of the scan kernel.
-// Decode + route (first kernel of the prefill scan): per (b, h, chunk) one block of
-// `chunk_bytes` holding the owner offsets, the owner-sorted event records and the write
-// retentions (layout: chunk_block_bytes()).
+// Event decode (first kernel of the prefill scan): every token's K write and K read events,
+// events[b][h][t][stream][j] = {slot, weight bits, alpha bits, t << 1 | stream}.
 struct RouteParams {
     const void* k_logits;  // [B,T,H,U*d_p]
     const void* q_logits;
@@ -35,18 +32,11 @@ struct RouteParams {
     int B, T, H;
     const int32_t* pos0;       // [B] or null
     const uint8_t* cape_mask;  // [H] or null
-    int ncta, cpl, chunk, nchunks;
-    int nwarps;             // scan warps per CTA (owners per CTA)
-    int chunks_per_block;   // set by the launcher
-    unsigned char* blocks;  // [B*H*nchunks][chunk_bytes]
-    size_t chunk_bytes, recs_off, alph_off;
-    float* o;               // [B,T,H,d_v] read accumulator, zeroed here
-    int d_v;
+    uint4* events;             // [B,H,T,2,K]
 };
 
 struct ScanParams {
-    const unsigned char* blocks;  // chunk blocks written by the route kernel
-    size_t chunk_bytes, recs_off, alph_off;
+    const uint4* events;  // [B,H,T,2,K] written by the event decode
     const void* v;  // [B,T,H,d_v]
     const void* z;  // [B,T,H,d_v]
     int in_bf16;
@@ -90,17 +80,13 @@ struct StepParams {
     float eps_gsu, eps_norm;
 };
 
-// Tensor-memory plan of the prefill scan: how many CTAs (cluster size) share one head's
-// slot array, the chunk length, and the TMEM columns and shared memory of each CTA.
-// Returns false if the slot array does not fit.
+// Tensor-memory plan of the prefill scan: how many CTAs share one head's slot array, the
+// chunk length, and the TMEM columns and shared memory of each CTA.  Returns false if the
+// slot array does not fit.
 bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* plan);
-// Bytes of one chunk block (offsets, records, retentions) and the offsets of its parts.
-size_t chunk_block_bytes(int chunk, int K, int ncta, int nwarps, size_t* recs_off, size_t* alph_off);
+
 
 cudaError_t launch_decode_addresses(const DecodeParams& p, cudaStream_t stream);
-// Shared memory of one decode/route block of G chunks (largest G: 64 / chunk).
-size_t route_smem_bytes(int chunk, int G, int K, int n_owners);
-int route_chunks_per_block(int chunk, int nchunks);
 cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream);
 // One block whose bounded wait on a never-signalled barrier runs out after limit_ns.

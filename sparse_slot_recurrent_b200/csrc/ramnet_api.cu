@@ -80,22 +80,19 @@ uint32_t* device_status_ptr()
     return static_cast<uint32_t*>(p);
 }
 
-// Scratch of the prefill scan: one block per (b, h, chunk) with the owner offsets, the
-// owner-sorted event records and the write retentions, then the fp32 read accumulator
-// [B,T,H,d_v] at a 256-byte boundary.
+// Scratch of the prefill scan: the decoded events [B,H,T,2,K] (16 bytes each), then the
+// fp32 read accumulator [B,T,H,d_v] at a 256-byte boundary.
 struct WorkspaceLayout {
-    size_t chunk_bytes, recs_off, alph_off, o_off, total;
-    int nchunks;
+    size_t o_off, o_bytes, total;
 };
 
-WorkspaceLayout workspace_layout(int B, int T, int H, int K, int d_v, const ramnet::ScanPlan& plan)
+WorkspaceLayout workspace_layout(int B, int T, int H, int K, int d_v, const ramnet::ScanPlan&)
 {
     WorkspaceLayout w;
-    w.nchunks = (T + plan.chunk - 1) / plan.chunk;
-    w.chunk_bytes = ramnet::chunk_block_bytes(plan.chunk, K, plan.ncta, plan.nwarps, &w.recs_off, &w.alph_off);
-    const size_t blocks = static_cast<size_t>(B) * H * w.nchunks * w.chunk_bytes;
-    w.o_off = (blocks + 255) & ~static_cast<size_t>(255);
-    w.total = w.o_off + static_cast<size_t>(B) * T * H * d_v * sizeof(float);
+    const size_t events = static_cast<size_t>(B) * H * T * 2 * K * 16;
+    w.o_off = (events + 255) & ~static_cast<size_t>(255);
+    w.o_bytes = static_cast<size_t>(B) * T * H * d_v * sizeof(float);
+    w.total = w.o_off + w.o_bytes;
     return w;
 }
 
@@ -197,18 +194,11 @@ ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     rp.H = H;
     rp.pos0 = pos0;
     rp.cape_mask = cape_mask;
-    rp.ncta = plan.ncta;
-    rp.cpl = plan.cpl;
-    rp.chunk = plan.chunk;
-    rp.nchunks = wl.nchunks;
-    rp.nwarps = plan.nwarps;
-    rp.blocks = static_cast<unsigned char*>(workspace);
-    rp.chunk_bytes = wl.chunk_bytes;
-    rp.recs_off = wl.recs_off;
-    rp.alph_off = wl.alph_off;
-    rp.o = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + wl.o_off);
-    rp.d_v = cfg->d_v;
-    cudaError_t e = ramnet::launch_decode_route(rp, s);
+    rp.events = static_cast<uint4*>(workspace);
+    // the read accumulator of the recurrence starts at zero
+    cudaError_t e = cudaMemsetAsync(static_cast<unsigned char*>(workspace) + wl.o_off, 0, wl.o_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: accumulator reset");
+    e = ramnet::launch_decode_route(rp, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan: decode/route launch");
     return RAMNET_OK;
 }
@@ -221,10 +211,7 @@ ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     uint32_t* status = device_status_ptr();
     if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
     ramnet::ScanParams sp{};
-    sp.blocks = static_cast<unsigned char*>(workspace);
-    sp.chunk_bytes = wl.chunk_bytes;
-    sp.recs_off = wl.recs_off;
-    sp.alph_off = wl.alph_off;
+    sp.events = static_cast<const uint4*>(workspace);
     sp.v = v;
     sp.z = z;
     sp.in_bf16 = in_dt == RAMNET_BF16;

@@ -13,12 +13,13 @@
 // columns [(s/4)*CPL, (s/4)*CPL + CPL); lane l of the quadrant holds channels
 // [l*CPL, l*CPL + CPL).  One slot row is one tcgen05.ld/st of CPL columns by a warp of
 // that quadrant.  Scan warp w (0..15) owns the local slots with s mod 16 == w and walks
-// their events, which the decode kernel has grouped per chunk of C tokens into one
-// token-ordered list per owner warp (writes before reads within a token).
+// their events in token order (a token's writes before its reads).
 //
-// Per CTA: a loader warp bulk-copies each chunk's event block and value rows into a ring
-// of kStages shared-memory stages; each scan warp walks its own list of every chunk at its
-// own pace (no barrier between scan warps; a stage is recycled once all 16 have left it):
+// Per CTA: a loader warp bulk-copies each chunk's events (C tokens, token order, as the
+// event decode wrote them) and value rows into a ring of kStages shared-memory stages;
+// each scan warp picks its own events out of the chunk 32 at a time (one ballot per 32
+// events) and walks them at its own pace (no barrier between scan warps; a stage is
+// recycled once all 16 have left it):
 //   write event  GSU steps 1-3 on the slot's mass (m = alpha*m + w, lambda = w/(m+eps),
 //                m kept in shared memory), step 4 on the row (tcgen05.ld, update,
 //                tcgen05.st);
@@ -51,14 +52,15 @@ __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~static_
 
 struct Layout {
     size_t bars, misc, m, stage, total;
-    size_t stage_bytes, blk_bytes, v_off;
+    size_t stage_bytes, v_off;
 };
 
-__host__ __device__ inline Layout scan_layout(int Ml, int C, int dv, int es, size_t chunk_bytes)
+// Shared memory of the scan kernel: barriers, masses of the CTA's slots, and kStages stages
+// of [C tokens x 2 streams x K events] 16-byte records followed by C value rows.
+__host__ __device__ inline Layout scan_layout(int Ml, int C, int K, int dv, int es)
 {
     Layout L;
-    L.blk_bytes = align16(chunk_bytes);
-    L.v_off = L.blk_bytes;
+    L.v_off = static_cast<size_t>(C) * 2 * K * sizeof(uint4);
     L.stage_bytes = L.v_off + align16(static_cast<size_t>(C) * dv * es);
     size_t o = 0;
     L.bars = o;
@@ -256,8 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Ml = (M - rank + ncta - 1) / ncta;
     const int nch = (p.T + C - 1) / C;
-    const int E = 2 * C * K;  // event capacity of a chunk; bounds every list walk
-    const Layout L = scan_layout((M + ncta - 1) / ncta, C, dv, es, p.chunk_bytes);
+    const int lg_ncta = __ffs(ncta) - 1;
+    const Layout L = scan_layout((M + ncta - 1) / ncta, C, K, dv, es);
     const uint32_t bars = smem_addr(smem + L.bars);
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
     uint64_t* bar_ptr = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -295,58 +297,54 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             tmem_st<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), r);
         }
         tmem_wait_st();
-        const int o_own = rank * kScanWarps + warp;
         for (int c = 0; c < nch; ++c) {
             wait_bounded(bar(kBarStage + c % kStages), (c / kStages) & 1, p.status, abort_flag);
             const unsigned char* st = stage(c);
-            const int* ofs = reinterpret_cast<const int*>(st);
-            const uint2* recs = reinterpret_cast<const uint2*>(st + p.recs_off);
-            const float* alph = reinterpret_cast<const float*>(st + p.alph_off);
+            const uint4* evs = reinterpret_cast<const uint4*>(st);
             const unsigned char* vb = st + L.v_off;
-            const int beg = min(max(ofs[o_own], 0), E);
-            const int end = min(max(ofs[o_own + 1], beg), E);
-            // o row of token t of this chunk
-            float* orow0 = p.o + ((static_cast<size_t>(b) * p.T + static_cast<size_t>(c) * C) * p.H + h) * dv + lch;
+            const int nev = min(C, p.T - c * C) * 2 * K;
+            const int t0 = c * C;
+            // o row of token t0 of this chunk; token t at + (t - t0) * H * d_v
+            float* orow0 = p.o + ((static_cast<size_t>(b) * p.T + t0) * p.H + h) * dv + lch;
             const size_t ostride = static_cast<size_t>(p.H) * dv;
-            uint2 nxt = beg < end ? recs[beg] : make_uint2(0u, 0u);
-            float vn[CPL];  // value row of event `nxt` (writes)
-            load_row<CPL>(vb, static_cast<int>(nxt.x >> 24) * dv + lch, p.in_bf16, vn);
-            for (int i = beg; i < end; ++i) {
-                const uint2 rec = nxt;
-                float vv[CPL];
+            for (int base = 0; base < nev; base += 32) {
+                const int e = base + lane;
+                const uint4 r = e < nev ? evs[e] : make_uint4(0u, 0u, 0u, 0u);
+                const int sloc = static_cast<int>(r.x >> lg_ncta);
+                const bool mine = e < nev && static_cast<int>(r.x & (ncta - 1)) == rank && (sloc & (kScanWarps - 1)) == warp;
+                uint32_t mask = __ballot_sync(0xffffffffu, mine);
+                while (mask != 0u) {
+                    const int src = __ffs(mask) - 1;
+                    mask &= mask - 1u;
+                    const int sl = __shfl_sync(0xffffffffu, sloc, src);
+                    const float cf = __uint_as_float(__shfl_sync(0xffffffffu, r.y, src));
+                    const float al = __uint_as_float(__shfl_sync(0xffffffffu, r.z, src));
+                    const uint32_t tag = __shfl_sync(0xffffffffu, r.w, src);
+                    const int tl = static_cast<int>(tag >> 1) - t0;
+                    const uint32_t col = static_cast<uint32_t>((sl >> 2) * CPL);
+                    float S[CPL];
+                    tmem_ld<CPL>(tq + col, S);
+                    if ((tag & 1u) == 0u) {
+                        // write: GSU steps 1-3, m = alpha*m + w, lambda = w / (m + eps); step 4
+                        float vv[CPL];
+                        load_row<CPL>(vb, tl * dv + lch, p.in_bf16, vv);
+                        const float mn = fmaf(al, m_s[sl], cf);
+                        const float lam = cf / (mn + p.eps_gsu);
+                        __syncwarp();
+                        if (lane == 0) m_s[sl] = mn;
+                        __syncwarp();
+                        tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < CPL; ++cc) vv[cc] = vn[cc];
-                const uint32_t col = rec.x & 0x3FFu;
-                const int t = static_cast<int>(rec.x >> 24);
-                const float cf = __uint_as_float(rec.y);
-                float S[CPL];
-                tmem_ld<CPL>(tq + col, S);
-                const bool wr = (rec.x & 0x8000u) != 0u;
-                float al = 1.0f;
-                if (wr) al = alph[i];
-                if (i + 1 < end) {
-                    nxt = recs[i + 1];
-                    load_row<CPL>(vb, static_cast<int>(nxt.x >> 24) * dv + lch, p.in_bf16, vn);
-                }
-                if (wr) {
-                    // GSU steps 1-3: m = alpha*m + w, lambda = w / (m + eps); step 4 on the row
-                    const int sl = 4 * static_cast<int>(col / CPL) + q;
-                    const float mn = fmaf(al, m_s[sl], cf);
-                    const float lam = cf / (mn + p.eps_gsu);
-                    __syncwarp();
-                    if (lane == 0) m_s[sl] = mn;
-                    __syncwarp();
-                    tmem_wait_ld();
+                        for (int cc = 0; cc < CPL; ++cc) S[cc] = fmaf(lam, vv[cc] - S[cc], S[cc]);
+                        tmem_st<CPL>(tq + col, S);
+                        tmem_wait_st();
+                    } else {
+                        // read: r * S into the token's read accumulator
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int cc = 0; cc < CPL; ++cc) S[cc] = fmaf(lam, vv[cc] - S[cc], S[cc]);
-                    tmem_st<CPL>(tq + col, S);
-                    tmem_wait_st();
-                } else {
-                    // read: r * S into the token's read accumulator
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int cc = 0; cc < CPL; ++cc) S[cc] *= cf;
-                    if (lane < LW) red_add_row<CPL>(orow0 + static_cast<size_t>(t) * ostride, S);
+                        for (int cc = 0; cc < CPL; ++cc) S[cc] *= cf;
+                        if (lane < LW) red_add_row<CPL>(orow0 + static_cast<size_t>(tl) * ostride, S);
+                    }
                 }
             }
             arrive_cta(bar(kBarFree + c % kStages));
@@ -366,7 +364,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
     } else {
         // ============================================================ loader warp
         const uint32_t vrow = static_cast<uint32_t>(dv * es);
-        const uint32_t blk = static_cast<uint32_t>(p.chunk_bytes);
         for (int c = 0; c < nch; ++c) {
             const int n = min(C, p.T - c * C);
             if (c >= kStages) {
@@ -375,10 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             }
             unsigned char* st = stage(c);
             const uint32_t sb = bar(kBarStage + c % kStages);
-            if (lane == 0) arrive_expect_tx(sb, blk + static_cast<uint32_t>(n) * vrow);
+            const uint32_t evb = static_cast<uint32_t>(n * 2 * K * sizeof(uint4));
+            if (lane == 0) arrive_expect_tx(sb, evb + static_cast<uint32_t>(n) * vrow);
             __syncwarp();
             if (lane == 0)
-                bulk_g2s(smem_addr(st), p.blocks + (static_cast<size_t>(bh) * nch + c) * p.chunk_bytes, blk, sb);
+                bulk_g2s(smem_addr(st), p.events + (static_cast<size_t>(bh) * p.T + static_cast<size_t>(c) * C) * 2 * K, evb,
+                         sb);
             for (int t = lane; t < n; t += 32) {
                 const size_t th = (static_cast<size_t>(b) * p.T + c * C + t) * p.H + h;
                 bulk_g2s(smem_addr(st + L.v_off + static_cast<size_t>(t) * vrow),
@@ -443,16 +442,6 @@ __global__ void k_wait_selftest(uint32_t* status, uint64_t limit_ns)
 
 }  // namespace
 
-size_t chunk_block_bytes(int chunk, int K, int ncta, int nwarps, size_t* recs_off, size_t* alph_off)
-{
-    const size_t E = static_cast<size_t>(2) * chunk * K;
-    const size_t ro = align16(sizeof(int) * (nwarps * ncta + 1));
-    const size_t ao = ro + align16(sizeof(uint2) * E);
-    if (recs_off) *recs_off = ro;
-    if (alph_off) *alph_off = ao;
-    return align16(ao + sizeof(float) * E);
-}
-
 bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
 {
     const int cpl = d_v < 32 ? 1 : d_v / 32;
@@ -470,15 +459,11 @@ bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
     const int cols = ((Ml + 3) / 4) * cpl;
     uint32_t alloc = 32;
     while (alloc < static_cast<uint32_t>(cols)) alloc <<= 1;
-    auto total = [&](int cc) {
-        return scan_layout(Ml, cc, d_v, in_bytes, chunk_block_bytes(cc, K, n, kScanWarps, nullptr, nullptr)).total;
-    };
-    // the decode/route kernel's block for the largest number of chunks per block
-    auto route = [&](int cc) { return route_smem_bytes(cc, route_chunks_per_block(cc, 1 << 30), K, n * kScanWarps); };
+    auto total = [&](int cc) { return scan_layout(Ml, cc, K, d_v, in_bytes).total; };
     const size_t budget = 200 * 1024;
     int C = 64;
-    while (C > 2 && (total(C) > budget || route(C) > budget)) C >>= 1;
-    if (total(C) > budget || route(C) > budget) return false;
+    while (C > 1 && total(C) > budget) C >>= 1;
+    if (total(C) > budget) return false;
     out->ncta = n;
     out->nwarps = kScanWarps;
     out->chunk = C;
