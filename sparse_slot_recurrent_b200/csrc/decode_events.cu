@@ -1,4 +1,4 @@
-// decode_route.cu -- K1 of the prefill scan: the Address Decoder and CAPE for every token
+// decode_events.cu -- K1 of the prefill scan: the Address Decoder and CAPE for every token
 // of every head, written as read and write events in token order.
 //
 // RAM-Net project page, GPU-execution paragraph: Top-K addresses for all tokens are
@@ -21,7 +21,7 @@ namespace {
 constexpr int kEventThreads = 128;
 
 template <int KMAX, int DPMAX>
-__global__ void __launch_bounds__(kEventThreads) k_decode_events(RouteParams p)
+__global__ void __launch_bounds__(kEventThreads) k_decode_events(EventParams p)
 {
     extern __shared__ uint64_t kept_s[];  // [KMAX][kEventThreads], K > 16 only
     const long long n = static_cast<long long>(p.B) * p.H * p.T * 2;
@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kEventThreads) k_decode_events(RouteParams p)
 }
 
 template <int KMAX, int DPMAX>
-cudaError_t launch_events(const RouteParams& p, cudaStream_t s)
+cudaError_t launch_events(const EventParams& p, cudaStream_t s)
 {
     const long long n = static_cast<long long>(p.B) * p.H * p.T * 2;
     const unsigned blocks = static_cast<unsigned>((n + kEventThreads - 1) / kEventThreads);
@@ -74,7 +74,7 @@ cudaError_t launch_events(const RouteParams& p, cudaStream_t s)
 }
 
 template <int DPMAX>
-cudaError_t events_k(const RouteParams& p, cudaStream_t s)
+cudaError_t events_k(const EventParams& p, cudaStream_t s)
 {
     if (p.K <= 8) return launch_events<8, DPMAX>(p, s);
     if (p.K <= 16) return launch_events<16, DPMAX>(p, s);
@@ -84,7 +84,7 @@ cudaError_t events_k(const RouteParams& p, cudaStream_t s)
 
 }  // namespace
 
-cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream)
+cudaError_t launch_decode_events(const EventParams& p, cudaStream_t stream)
 {
     if (p.T >= (1 << 30)) return cudaErrorInvalidValue;
     if (p.d_p <= 4) return events_k<4>(p, stream);

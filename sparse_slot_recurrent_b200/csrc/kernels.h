@@ -23,7 +23,7 @@ struct DecodeParams {
 
 // Event decode (first kernel of the prefill scan): every token's K write and K read events,
 // events[b][h][t][stream][j] = {slot, weight bits, alpha bits, t << 1 | stream}.
-struct RouteParams {
+struct EventParams {
     const void* k_logits;  // [B,T,H,U*d_p]
     const void* q_logits;
     const void* g;  // [B,T,H]
@@ -53,7 +53,7 @@ struct ScanParams {
     float eps_gsu, eps_norm;
     uint32_t tmem_cols;
     uint32_t* status;
-    float* o;  // [B,T,H,d_v] read accumulator (zeroed by the route kernel)
+    float* o;  // [B,T,H,d_v] read accumulator (reset to zero by ramnet_scan_route)
 };
 
 struct ScanPlan {
@@ -87,7 +87,7 @@ bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* plan);
 
 
 cudaError_t launch_decode_addresses(const DecodeParams& p, cudaStream_t stream);
-cudaError_t launch_decode_route(const RouteParams& p, cudaStream_t stream);
+cudaError_t launch_decode_events(const EventParams& p, cudaStream_t stream);
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream);
 // One block whose bounded wait on a never-signalled barrier runs out after limit_ns.
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);

@@ -179,7 +179,7 @@ ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
                          const void* q_logits, const void* g, const uint8_t* cape_mask, const int32_t* pos0,
                          void* workspace, cudaStream_t s)
 {
-    ramnet::RouteParams rp{};
+    ramnet::EventParams rp{};
     rp.k_logits = k_logits;
     rp.q_logits = q_logits;
     rp.g = g;
@@ -198,8 +198,8 @@ ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     // the read accumulator of the recurrence starts at zero
     cudaError_t e = cudaMemsetAsync(static_cast<unsigned char*>(workspace) + wl.o_off, 0, wl.o_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan: accumulator reset");
-    e = ramnet::launch_decode_route(rp, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan: decode/route launch");
+    e = ramnet::launch_decode_events(rp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: event decode launch");
     return RAMNET_OK;
 }
 

@@ -11,11 +11,12 @@
 // RAMNET_NOALLOC_SCRATCH_BYTES bytes, 256-byte aligned.  The first call on a device (that
 // device being current) looks up the array's device address with cudaGetSymbolAddress
 // and caches it; later calls on that device reuse the cached address.  The call then runs
-// the same decode/route and scan kernels as ramnet_scan_forward with that address as the
+// the same event-decode and scan kernels as ramnet_scan_forward with that address as the
 // workspace.  Nothing here, or in what it calls, allocates device or host memory.
 //
-// Contents: nothing in the array has to start at zero.  Each call's decode/route kernel
-// writes every byte of the workspace that the same call's scan kernel later reads.
+// Contents: nothing in the array has to start at zero.  Each call writes every event the
+// scan reads (event decode) and resets the read accumulator itself before the scan adds
+// into it.
 //
 // Sharing: there is one array per device and per loaded copy of the library.  Two calls
 // whose kernels can be in flight at the same time (different streams, or different host
