@@ -307,9 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             // o row of token t0 of this chunk; token t at + (t - t0) * H * d_v
             float* orow0 = p.o + ((static_cast<size_t>(b) * p.T + t0) * p.H + h) * dv + lch;
             const size_t ostride = static_cast<size_t>(p.H) * dv;
+            uint4 rn = lane < nev ? evs[lane] : make_uint4(0u, 0u, 0u, 0u);  // next group, prefetched
             for (int base = 0; base < nev; base += 32) {
                 const int e = base + lane;
-                const uint4 r = e < nev ? evs[e] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 r = rn;
+                if (base + 32 < nev) rn = e + 32 < nev ? evs[e + 32] : make_uint4(0u, 0u, 0u, 0u);
                 const int sloc = static_cast<int>(r.x >> lg_ncta);
                 const bool mine = e < nev && static_cast<int>(r.x & (ncta - 1)) == rank && (sloc & (kScanWarps - 1)) == warp;
                 uint32_t mask = __ballot_sync(0xffffffffu, mine);
