@@ -331,10 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
                         float vv[CPL];
                         load_row<CPL>(vb, tl * dv + lch, p.in_bf16, vv);
                         const float mn = fmaf(al, m_s[sl], cf);
-                        const float lam = cf / (mn + p.eps_gsu);
-                        __syncwarp();
-                        if (lane == 0) m_s[sl] = mn;
-                        __syncwarp();
+                        const float lam = __fdividef(cf, mn + p.eps_gsu);
+                        m_s[sl] = mn;  // every lane stores the same value and later reads its own store
                         tmem_wait_ld();
 #pragma unroll
                         for (int cc = 0; cc < CPL; ++cc) S[cc] = fmaf(lam, vv[cc] - S[cc], S[cc]);
