@@ -97,11 +97,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# host-only sources of the library: they launch the kernels but hold no device code
+HOST_ONLY_SOURCES = ("ramnet_api.cu", "scan_noalloc.cu")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the device-code sources (a profile's counters apply while it is unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_slot_recurrent_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
+        if name.endswith((".cu", ".cuh", ".h")) and name not in HOST_ONLY_SOURCES:
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())

@@ -43,9 +43,9 @@
  *     returns RAMNET_ERR_INVALID_ARG or RAMNET_ERR_UNSUPPORTED and launches nothing.
  *     A launch error returns RAMNET_ERR_CUDA.  ramnet_last_error() describes the last
  *     failure of the calling thread.
- *   - Kernels that wait on other thread blocks wait a bounded number of iterations; when
- *     a wait gives up the kernel records it in a device status word and returns early.
- *     ramnet_sync_status() reads (and clears) that word.
+ *   - Where warps of a kernel wait for one another (the prefill scan's staging ring) every
+ *     wait is bounded (about 2 s); when a wait gives up the kernel records it in a device
+ *     status word and finishes early.  ramnet_sync_status() reads (and clears) that word.
  *   - No call allocates device memory.  Scratch space comes from the caller
  *     (ramnet_scan_forward's workspace) or, for ramnet_scan_forward_noalloc, from a
  *     fixed array inside the library's device image.
@@ -108,8 +108,9 @@ ramnet_status ramnet_decode_addresses(const ramnet_config* cfg, int32_t B, int32
                                       void* stream);
 
 /*
- * ramnet_scan_workspace_bytes -- scratch bytes ramnet_scan_forward needs for these sizes
- * (the decoded addresses of both streams).  Returns 0 for invalid arguments.
+ * ramnet_scan_workspace_bytes -- scratch bytes ramnet_scan_forward needs for these sizes:
+ * the decoded read and write events (32*K bytes per token-head) and an fp32 read
+ * accumulator (4*d_v bytes per token-head).  Returns 0 for invalid arguments.
  */
 size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H);
 
@@ -155,7 +156,9 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
  *   ramnet_scan_forward; writes the workspace (contents on entry ignored).
  * ramnet_scan_recur: the recurrence (GSU steps 1-4, sparse read after the token's write,
  *   RMSNorm, norm weight, output gate) over the events in the workspace, which must hold
- *   what ramnet_scan_route wrote for the same arguments; the workspace is only read.
+ *   what ramnet_scan_route wrote for the same arguments.  It adds the reads into the
+ *   workspace's read accumulator, which ramnet_scan_route resets: run it exactly once
+ *   after each ramnet_scan_route.
  *   v, z, norm_w, S_in, m_in, y, S_out, m_out as in ramnet_scan_forward.
  * Errors: as ramnet_scan_forward.
  */
@@ -167,7 +170,7 @@ ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, 
                                 ramnet_dtype in_dt, const void* v, const void* z,
                                 const float* norm_w, const float* S_in, const float* m_in, void* y,
                                 ramnet_dtype out_dt, float* S_out, float* m_out,
-                                const void* workspace, size_t workspace_bytes, void* stream);
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* Size of the scratch array built into the library for ramnet_scan_forward_noalloc. */
 #define RAMNET_NOALLOC_SCRATCH_BYTES ((size_t)32 * 1024 * 1024)

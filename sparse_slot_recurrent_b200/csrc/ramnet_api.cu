@@ -299,7 +299,7 @@ ramnet_status ramnet_scan_route(const ramnet_config* cfg, int32_t B, int32_t T, 
 ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
                                 const void* v, const void* z, const float* norm_w, const float* S_in,
                                 const float* m_in, void* y, ramnet_dtype out_dt, float* S_out, float* m_out,
-                                const void* workspace, size_t workspace_bytes, void* stream)
+                                void* workspace, size_t workspace_bytes, void* stream)
 {
     g_last_error.clear();
     int M = 0;
@@ -317,7 +317,7 @@ ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, 
     OPTIONAL_PTR(S_in);
     OPTIONAL_PTR(m_in);
     return recur_part(cfg, B, T, H, in_dt, M, plan, wl, v, z, norm_w, S_in, m_in, y, out_dt, S_out, m_out,
-                      const_cast<void*>(workspace), static_cast<cudaStream_t>(stream));
+                      workspace, static_cast<cudaStream_t>(stream));
 }
 
 ramnet_status ramnet_selftest_wait_timeout(uint32_t limit_us, void* stream)
