@@ -48,7 +48,7 @@ struct ScanParams {
     float* S_out;  // [B,H,M,d_v]
     float* m_out;  // [B,H,M]
     int B, T, H, K, M, d_v;
-    int ncta;   // CTAs per (b,h) = cluster size
+    int ncta;   // CTAs per (b,h); CTA r holds the slots i with i mod ncta == r
     int chunk;  // tokens per chunk
     float eps_gsu, eps_norm;
     uint32_t tmem_cols;
@@ -57,7 +57,7 @@ struct ScanParams {
 };
 
 struct ScanPlan {
-    int ncta, chunk, cpl, nchunks, nwarps;
+    int ncta, chunk, cpl;
     uint32_t tmem_cols;
     size_t smem_bytes;
 };

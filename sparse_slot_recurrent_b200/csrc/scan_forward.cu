@@ -24,8 +24,9 @@
 //                m kept in shared memory), step 4 on the row (tcgen05.ld, update,
 //                tcgen05.st);
 //   read event   the weighted row r*S is added into the token's read accumulator o
-//                [B,T,H,d_v] fp32 in global memory (vector red.add), which the decode
-//                kernel zeroed.  The read of token t follows t's own writes in the list.
+//                [B,T,H,d_v] fp32 in global memory (vector red.add), which
+//                ramnet_scan_route reset to zero.  The read of token t follows t's own
+//                writes in the list.
 // K2b then turns o into y: RMSNorm over d_v, norm weight, output gate.  The read
 // accumulator adds up to K terms per element in an order that can change from run to
 // run, so y may differ between runs in the last bits.
@@ -465,14 +466,12 @@ bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
     while (C > 1 && total(C) > budget) C >>= 1;
     if (total(C) > budget) return false;
     out->ncta = n;
-    out->nwarps = kScanWarps;
     out->chunk = C;
     out->cpl = cpl;
     out->tmem_cols = alloc;
     // more than half of the SM's shared memory: exactly one CTA (and one TMEM owner) per SM
     const size_t t = total(C);
     out->smem_bytes = t < 116 * 1024 ? 116 * 1024 : t;
-    out->nchunks = 0;
     return true;
 }
 
