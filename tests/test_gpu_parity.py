@@ -190,6 +190,20 @@ def test_scan_matches_oracle(case):
     assert _maxabs(m, om) <= tol
 
 
+def test_scan_raw_product_softmax_weights():
+    """renorm = 0 (weights are the raw truncated product softmax) through the whole scan."""
+    w, inp = _small_inputs(4, 5, 8, 64, 1, 150, 2, torch.float32, "mixed", seed=31)
+    cfg, ocfg = _cfgs(w, renorm=0)
+    g = torch.Generator().manual_seed(32)
+    S_in = torch.randn((1, 2, w.M, 64), generator=g)
+    m_in = torch.rand((1, 2, w.M), generator=g)
+    y, S, m = _gpu_scan(cfg, inp, None, S_in, m_in)
+    oy, oS, om = _oracle_scan(ocfg, inp, None, S_in, m_in)
+    assert _maxabs(y, oy) <= TOL_F32
+    assert _maxabs(S, oS) <= TOL_F32
+    assert _maxabs(m, om) <= TOL_F32
+
+
 def test_scan_route_then_recur_matches_oracle_and_forward():
     """The two-launch form (route, then recurrence over the workspace) gives the oracle's
     results and the single-call results (the state exactly)."""
