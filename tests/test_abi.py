@@ -122,3 +122,31 @@ def test_valid_call_without_device_reports_cuda_error(lib):
     # arguments pass every host check; with no device the first CUDA call fails cleanly
     assert _decode(lib, _cfg()) == ramnet.RAMNET_ERR_CUDA
     assert ramnet.last_error() != ""
+
+
+def test_scan_workspace_is_events_then_accumulator(lib):
+    # decoded events (16 bytes each, 2*K per token-head), then the fp32 read accumulator
+    # at a 256-byte boundary
+    for (d_p, U, K, d_v), (B, T, H) in [((4, 5, 8, 128), (8, 4096, 8)), ((3, 5, 7, 32), (1, 77, 2)),
+                                         ((16, 2, 64, 256), (2, 33, 3))]:
+        c = _cfg(d_p=d_p, U=U, K=K, d_v=d_v)._c()
+        events = B * H * T * 2 * K * 16
+        o_off = (events + 255) // 256 * 256
+        assert lib.ramnet_scan_workspace_bytes(ctypes.byref(c), B, T, H) == o_off + B * T * H * d_v * 4
+
+
+def test_two_launch_form_checks(lib):
+    cfg = _cfg()
+    c = cfg._c()
+    B, T, H = 2, 8, 2
+    need = lib.ramnet_scan_workspace_bytes(ctypes.byref(c), B, T, H)
+    route = lambda k=FAKE, ws=FAKE, n=need: lib.ramnet_scan_route(
+        ctypes.byref(c), B, T, H, ramnet.RAMNET_BF16, k, FAKE, FAKE, None, None, ws, n, None)
+    recur = lambda v=FAKE, ws=FAKE, n=need, od=ramnet.RAMNET_F32: lib.ramnet_scan_recur(
+        ctypes.byref(c), B, T, H, ramnet.RAMNET_BF16, v, FAKE, None, None, None, FAKE, od, FAKE, FAKE, ws, n, None)
+    assert route(k=None) == ramnet.RAMNET_ERR_INVALID_ARG and "k_logits" in ramnet.last_error()
+    assert route(n=need - 1) == ramnet.RAMNET_ERR_INVALID_ARG and "workspace" in ramnet.last_error()
+    assert route(ws=FAKE + 8) == ramnet.RAMNET_ERR_INVALID_ARG and "aligned" in ramnet.last_error()
+    assert recur(v=None) == ramnet.RAMNET_ERR_INVALID_ARG and "v" in ramnet.last_error()
+    assert recur(od=5) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert recur(ws=None) == ramnet.RAMNET_ERR_INVALID_ARG
