@@ -226,19 +226,19 @@ def weak_scaling_value(tokens_per_rank: int, world: int, max_ms: float) -> float
 
 # ------------------------------------------------------------------ oracle (CPU) timing
 
-def oracle_sample(w, n_heads: int, threads: int):
-    """Run the CPU oracle on the first n_heads (b,h) heads (whole sequences) of the
-    workload; returns (seconds, token-heads processed)."""
+def oracle_sample(w, n_heads: int, threads: int, T: int | None = None):
+    """Run the CPU oracle on the first n_heads (b,h) heads of the workload, over the first
+    T tokens (whole sequences by default); returns (seconds, token-heads processed)."""
     import oracle
     oracle.build()
     nb = max(1, (n_heads + w.H - 1) // w.H)
-    sub = w.with_(B=nb)
+    sub = w.with_(B=nb, T=T or w.T)
     inp = generate(sub, seed=0)
     ocfg = oracle.OracleConfig(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
     t0 = time.perf_counter()
     oracle.scan_forward(ocfg, inp["k_logits"], inp["q_logits"], inp["v"], inp["g"], inp["z"],
                         cape_mask=inp["cape_mask"], pos0=inp["pos0"], nthreads=threads)
-    return time.perf_counter() - t0, nb * w.H * w.T
+    return time.perf_counter() - t0, nb * w.H * sub.T
 
 
 def cpu_baseline(w, cores: int):
@@ -257,17 +257,23 @@ def run_reference(args, world, rank):
     w = WORKLOADS[PREFILL]
     cores = os.cpu_count() or 1
     n_heads = min(w.B * w.H, cores)
+    # keep the timed steps to about two minutes: shorten the sequences of each step's sample
+    # when whole sequences would take longer
+    t_step = None
     for _ in range(args.warmup):
-        oracle_sample(w, n_heads, cores)
+        t_step, _ = oracle_sample(w, n_heads, cores)
+    T = w.T
+    if t_step is not None and t_step * args.steps > 120.0:
+        T = max(64, int(w.T * 120.0 / (t_step * args.steps)))
     secs = []
     th = 0
     for _ in range(args.steps):
-        s, th = oracle_sample(w, n_heads, cores)
+        s, th = oracle_sample(w, n_heads, cores, T=T)
         secs.append(s)
     ms = 1e3 * statistics.mean(secs)
     value = th / w.H / (ms / 1e3)
     heads = ((n_heads + w.H - 1) // w.H) * w.H
-    sample = f"{heads} (b,h) heads x T={w.T} tokens of {w.name} per step"
+    sample = f"{heads} (b,h) heads x the first {T} of T={w.T} tokens of {w.name} per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
