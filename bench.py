@@ -2,14 +2,18 @@
 """Benchmark of the B200 RAM-Net layer core.
 
 One step = one ``ramnet_scan_forward`` call (address decode of keys and queries, CAPE,
-Gated Sparse Update, sparse read, RMSNorm, gate) over the 340M-like Top-8 prefill
-workload: B=8 sequences x T=4096 tokens x H=8 heads, d_p=4, U=5 (M=1024 slots), K=8,
-d_v=128, bf16 inputs and output, fp32 slot state, zero initial state.  Inputs are
-resident in HBM when timing starts; L2 is flushed (256 MiB write) between timed steps.
+Gated Sparse Update, sparse read, RMSNorm, gate), made as its two launches.  The headline
+workload is the 1.3B-like Top-16 long-context prefill: B=4 sequences x T=16384 tokens x
+H=16 heads, d_p=4, U=5 (M=1024 slots), K=16, d_v=128, CAPE on, bf16 inputs and output,
+fp32 slot state, zero initial state.  The 340M-like Top-8 and Top-32 prefills are timed
+the same way and reported under "prefill".  Inputs are resident in HBM when timing starts;
+L2 is flushed (256 MiB write) between timed steps.
 
 The JSON line also carries:
-  roofline     algorithmic bytes of the step / device time, against the measured HBM copy
-               bandwidth (MEASURED_PEAKS.json);
+  roofline     algorithmic bytes of the recurrence launch / its device time, against the
+               measured HBM copy bandwidth (MEASURED_PEAKS.json);
+  onchip       the slot-state bytes the recurrence moves through tensor memory (12*K*d_v per
+               token-head) / its device time, against the measured tensor-memory bandwidth;
   e2e          the same metric through the public API with pinned host buffers (H2D of the
                step's inputs and D2H of y inside the timed region);
   decode       the batched decode step (B=256, H=16, M=4096, K=16, d_v=128, state resident
@@ -44,7 +48,14 @@ import torch  # noqa: E402
 from sparse_slot_recurrent_b200.workloads import WORKLOADS, generate  # noqa: E402
 
 METRIC = "RAM-Net layer tokens/s (prefill scan, decode step) and % of HBM roofline"
-PREFILL = "prefill_340m_top8"
+# the largest prefill configuration is the headline; the other two are timed beside it
+PREFILL = "prefill_1p3b_top16"
+PREFILL_ALL = ("prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16")
+LAUNCHES_PER_STEP = 2  # route (k_route) and recurrence (k_scan)
+SM_COUNT = 148
+# tensor-memory bytes per clock per SM (32x32b.x4 load and store, many warps, batched waits),
+# measured on this machine; the on-chip roofline denominator
+TMEM_BYTES_PER_CLK_SM = 120.0
 DECODE = "decode_b256"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
@@ -254,7 +265,7 @@ def run_reference(args, world, rank):
     """The reference arm: the CPU oracle, timed on the host cores, rank 0 only."""
     if rank != 0:
         return
-    w = WORKLOADS[PREFILL]
+    w = WORKLOADS[args.workload]
     cores = os.cpu_count() or 1
     n_heads = min(w.B * w.H, cores)
     # keep the timed steps to about two minutes: shorten the sequences of each step's sample
@@ -294,10 +305,16 @@ def config_of(w, world):
 
 # ------------------------------------------------------------------ GPU arm
 
-def run_gpu(args, world, rank, local):
+def onchip_state_bytes(w) -> int:
+    """State bytes the recurrence moves on chip per launch: per token-head K write rows read
+    and written and K read rows read (fp32, 12*K*d_v bytes)."""
+    return w.B * w.T * w.H * 12 * w.K * w.d_v
+
+
+def time_prefill(args, world, rank, local, w, with_e2e: bool):
+    """Time the prefill step (route + recurrence, the two launches ramnet_scan_forward makes)
+    on workload w; returns the per-workload object of the JSON line."""
     from sparse_slot_recurrent_b200 import ramnet
-    ramnet.load()
-    w = WORKLOADS[args.workload]
     cfg = ramnet.Config(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
     dev = torch.device("cuda", local)
     inp = generate(w, seed=rank)
@@ -310,6 +327,7 @@ def run_gpu(args, world, rank, local):
     ws = torch.empty(ramnet.scan_workspace_bytes(cfg, w.B, w.T, w.H), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    lay = ramnet.scan_layout(cfg, w.in_dtype)
 
     def route():
         ramnet.scan_route(cfg, d["k_logits"], d["q_logits"], d["g"], ws, cape_mask=d["cape_mask"], pos0=d["pos0"],
@@ -322,7 +340,6 @@ def run_gpu(args, world, rank, local):
         route()
         recur()
 
-    launches_per_step = 3  # event decode; recurrence and output normalisation (plus one memset)
     for _ in range(args.warmup):
         step()
     ramnet.sync_status(stream)
@@ -349,30 +366,39 @@ def run_gpu(args, world, rank, local):
     tokens = w.B * w.T
     value = weak_scaling_value(tokens, world, ms_max)
 
-    # roofline of the dominant kernel (the recurrence) against measured HBM bandwidth,
-    # plus the same figures for the address launch and the whole step
+    # roofline of the dominant kernel (the recurrence) against measured HBM bandwidth, plus
+    # the same figures for the address launch and the whole step
     peak, peak_kind = measured_peaks()
     nb = 2 if w.in_dtype == torch.bfloat16 else 4
     alg_recur = recur_algorithmic_bytes(w, in_bytes=nb, out_bytes=nb)
     alg_route = route_algorithmic_bytes(w, in_bytes=nb)
     alg = prefill_algorithmic_bytes(w, in_bytes=nb, out_bytes=nb)
     achieved = alg_recur / (recur_ms / 1e3) / 1e9
-    traffic = recorded_traffic("recur")
+    traffic = recorded_traffic(f"recur:{w.name}")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
-                "kernel": "k_scan + k_scan_norm (ramnet_scan_recur)", "algorithmic_bytes": alg_recur,
+                "kernel": "k_scan (ramnet_scan_recur)", "algorithmic_bytes": alg_recur,
                 "ms_per_launch": recur_ms, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"}
+    # on-chip: the slot state the recurrence reads and writes (tensor memory), against the
+    # tensor-memory bandwidth measured on this machine at the sampled SM clock
+    sm_mhz = clk["sm_mhz"] if clk else 1965.0
+    ctas = w.B * w.H * lay.ncta
+    onchip_peak = TMEM_BYTES_PER_CLK_SM * min(ctas, SM_COUNT) * sm_mhz * 1e6 / 1e9
+    onchip_ach = onchip_state_bytes(w) / (recur_ms / 1e3) / 1e9
+    onchip = {"bytes_per_token_head": 12 * w.K * w.d_v, "achieved": onchip_ach, "peak": onchip_peak, "unit": "GB/s",
+              "frac": onchip_ach / onchip_peak, "sm_mhz": sm_mhz, "sms_used": min(ctas, SM_COUNT),
+              "peak_basis": f"{TMEM_BYTES_PER_CLK_SM} B/clk/SM tensor-memory load+store probe x SMs x SM clock"}
     kernels = {
-        "route (memset + k_decode_events)": {"ms": route_ms, "algorithmic_bytes": alg_route,
-                                             "achieved_gbs": alg_route / (route_ms / 1e3) / 1e9},
-        "recur (k_scan + k_scan_norm)": {"ms": recur_ms, "algorithmic_bytes": alg_recur, "achieved_gbs": achieved},
+        "route (k_route)": {"ms": route_ms, "algorithmic_bytes": alg_route,
+                            "achieved_gbs": alg_route / (route_ms / 1e3) / 1e9},
+        "recur (k_scan)": {"ms": recur_ms, "algorithmic_bytes": alg_recur, "achieved_gbs": achieved},
         "step": {"ms": ms, "algorithmic_bytes": alg, "achieved_gbs": alg / (ms / 1e3) / 1e9,
                  "frac": alg / (ms / 1e3) / 1e9 / peak},
     }
 
     # end to end through the public API from pinned host memory
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
         keys = ("k_logits", "q_logits", "v", "g", "z", "cape_mask", "pos0")
         yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
         h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
@@ -387,10 +413,10 @@ def run_gpu(args, world, rank, local):
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(dev)
-        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+        n_e2e = max(3, min(args.steps, 20))
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
         dist_barrier(world)
-        for i in range(args.steps):
+        for i in range(n_e2e):
             flush.zero_()
             ee[i][0].record(stream)
             e2e_step()
@@ -398,19 +424,35 @@ def run_gpu(args, world, rank, local):
         torch.cuda.synchronize(dev)
         e_ms = dist_max(statistics.mean(a.elapsed_time(b) for a, b in ee), world)
         e2e = {"value": weak_scaling_value(tokens, world, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": n_e2e}
+    del flush, ws, y, S, m, d
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "config": config_of(w, world), "value": value, "unit": "tokens/s",
+            "ms_per_step": ms_max, "steps": args.steps, "roofline": roofline, "onchip": onchip, "kernels": kernels,
+            "e2e": e2e, "clocks": clk, "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "plan": {"chunk": lay.chunk, "ctas_per_head": lay.ncta, "scan_warps": lay.scan_warps}}
 
+
+def run_gpu(args, world, rank, local):
+    from sparse_slot_recurrent_b200 import ramnet
+    ramnet.load()
+    head = WORKLOADS[args.workload]
+    others = [] if args.only_headline else [n for n in PREFILL_ALL if n != head.name]
+    main = time_prefill(args, world, rank, local, head, with_e2e=not args.no_e2e)
+    prefill = {head.name: {k: v for k, v in main.items() if k != "e2e"}}
+    for name in others:
+        prefill[name] = time_prefill(args, world, rank, local, WORKLOADS[name], with_e2e=False)
     decode = None if args.no_decode else run_decode(args, world, local)
-    del flush
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; shapes of the 340M-like layer)",
-                "config": config_of(w, world), "roofline": roofline, "kernels": kernels, "e2e": e2e,
-                "gpu_launches": launches_per_step * args.steps, "clocks": clk, "decode": decode}
+        line = {"metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded; shapes of the 340M / 1.3B layers)", "config": main["config"],
+                "roofline": main["roofline"], "onchip": main["onchip"], "kernels": main["kernels"], "e2e": main["e2e"],
+                "gpu_launches": main["gpu_launches"], "clocks": main["clocks"], "prefill": prefill, "decode": decode}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, os.cpu_count() or 1)
+            line["cpu_baseline"] = cpu_baseline(head, os.cpu_count() or 1)
         print(json.dumps(line), flush=True)
 
 
@@ -480,7 +522,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ramnet", "reference"], default="ramnet")
     ap.add_argument("--workload", default=PREFILL, choices=[k for k, v in WORKLOADS.items() if not v.decode],
-                    help="prefill workload of the timed step (default: the 340M-like Top-8 layer)")
+                    help="headline prefill workload (default: the 1.3B-like Top-16 long-context layer)")
+    ap.add_argument("--only-headline", action="store_true", help="time only the headline prefill workload")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -89,30 +89,66 @@ typedef struct {
     int32_t renorm;   /* 1: weights renormalised over the K selected slots */
 } ramnet_config;
 
+/* Element strides of a [B,T,H,L] logits array whose last dimension is contiguous: element
+ * (b, t, h, l) sits at b*b_stride + t*t_stride + h*h_stride + l.  Strides are >= 0 and may
+ * describe a permuted or sliced view (for example a [B,H,T,L] array read as [B,T,H,L]). */
+typedef struct {
+    int64_t b, t, h;
+} ramnet_strides;
+
 /*
  * ramnet_decode_addresses -- Address Decoder and CAPE for a batch of tokens.
  * Project page: Product Softmax paragraph, the five views (exact Top-K search in the
  * Multilevel Decision Tree view and the exactness paragraph after them), CAPE paragraphs.
  *
- *   logits    [B,T,H,U*d_p]  dtype `dt` (RAMNET_F32 or RAMNET_BF16)
+ *   logits    [B,T,H,U*d_p]  dtype `dt` (RAMNET_F32 or RAMNET_BF16), laid out as `strides`
+ *             says (NULL: dense, strides (T*H*L, H*L, L)); only element alignment is needed
  *   pos0      [B] int32 start position of each sequence, or NULL (all 0)
  *   cape_mask [H] uint8, nonzero = CAPE on for that head, or NULL (CAPE off)
- *   idx_out   [B,T,H,K] int32: selected slot indices, best first, after CAPE
- *   w_out     [B,T,H,K] fp32: their weights (same order)
- * Errors: INVALID_ARG for null logits/outputs, non-positive sizes, misalignment or a
- * config outside the limits.
+ *   idx_out   [B,T,H,K] int32 (dense): selected slot indices, best first, after CAPE
+ *   w_out     [B,T,H,K] fp32 (dense): their weights (same order)
+ * Errors: INVALID_ARG for null logits/outputs, non-positive sizes, a negative stride,
+ * misalignment or a config outside the limits.
  */
 ramnet_status ramnet_decode_addresses(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
-                                      const void* logits, ramnet_dtype dt, const int32_t* pos0,
-                                      const uint8_t* cape_mask, int32_t* idx_out, float* w_out,
-                                      void* stream);
+                                      const void* logits, ramnet_dtype dt, const ramnet_strides* strides,
+                                      const int32_t* pos0, const uint8_t* cape_mask, int32_t* idx_out,
+                                      float* w_out, void* stream);
 
 /*
- * ramnet_scan_workspace_bytes -- scratch bytes ramnet_scan_forward needs for these sizes:
- * the decoded read and write events (32*K bytes per token-head) and an fp32 read
- * accumulator (4*d_v bytes per token-head).  Returns 0 for invalid arguments.
+ * ramnet_scan_workspace_bytes -- scratch bytes ramnet_scan_forward needs for these sizes
+ * (the larger of the fp32- and bf16-input plans): the decoded read and write events
+ * (16 bytes each, 2*K per token, grouped per chunk of tokens) and a small header per
+ * (head, chunk, CTA rank); see ramnet_scan_layout.  Returns 0 for invalid arguments.
  */
 size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H);
+
+/*
+ * ramnet_scan_layout -- how ramnet_scan_forward splits the work for this config and input
+ * dtype, which fixes the workspace contents after ramnet_scan_route.  The pages have no
+ * counterpart: it serves tools and tests that read the workspace.
+ *
+ *   *chunk       tokens per chunk C (nch = ceil(T / C) chunks per head)
+ *   *ncta        CTAs per head (one thread-block cluster); slot i belongs to rank i mod ncta
+ *                as local slot s = i / ncta
+ *   *scan_warps  scan warps per CTA (nw); local slot s belongs to scan warp s mod nw
+ *   *hdr_words   32-bit words per (head, chunk, rank) header
+ *
+ * Workspace contents after ramnet_scan_route (head = b*H + h):
+ *   events at offset 0: [B*H][nch][2*C*K] records of 4 uint32 {x, weight, alpha, slot}; a
+ *     chunk's records are sorted by owner (rank * nw + scan warp) and, within one owner, by
+ *     (token, stream).  x = s | tl << 16 | q << 24 | stream << 31 with s the local slot, tl
+ *     the token within the chunk, stream 0 for a write (key) and 1 for a read (query), q
+ *     the read's rank among the token's reads held by the same rank; weight and alpha are
+ *     f32 bits (alpha = the write's retention, 0 for reads); slot is the index after CAPE.
+ *   headers at offset round_up(B*H*nch*2*C*K*16, 256): [B*H][nch][ncta][hdr_words] uint32:
+ *     [0] first record of the rank in the chunk, [1] the rank's record count, [2] tokens
+ *     in the chunk, [3] 0, [4 + w] (w = 0..nw) start of scan warp w's records relative to
+ *     [0], then one byte per token: how many of its reads the rank holds.
+ * Errors: INVALID_ARG (config, dtype, NULL outputs), UNSUPPORTED as ramnet_scan_forward.
+ */
+ramnet_status ramnet_scan_layout(const ramnet_config* cfg, ramnet_dtype in_dt, int32_t* chunk, int32_t* ncta,
+                                 int32_t* scan_warps, int32_t* hdr_words);
 
 /*
  * ramnet_scan_forward -- prefill: the whole layer core over T tokens, per (b,h) in token
@@ -153,12 +189,13 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
  *   retentions of GSU step 1, and the grouping of all read and write events by the scan
  *   warp that owns their slot (GPU-execution paragraph: addresses for all tokens first,
  *   events grouped by slot).  Reads k_logits, q_logits, g, cape_mask, pos0 as in
- *   ramnet_scan_forward; writes the workspace (contents on entry ignored).
+ *   ramnet_scan_forward; writes the workspace (contents on entry ignored; layout in
+ *   ramnet_scan_layout).
  * ramnet_scan_recur: the recurrence (GSU steps 1-4, sparse read after the token's write,
  *   RMSNorm, norm weight, output gate) over the events in the workspace, which must hold
- *   what ramnet_scan_route wrote for the same arguments.  It adds the reads into the
- *   workspace's read accumulator, which ramnet_scan_route resets: run it exactly once
- *   after each ramnet_scan_route.
+ *   what ramnet_scan_route wrote for the same arguments.  It only reads the workspace, so
+ *   it may run more than once after one ramnet_scan_route (same results each time: every
+ *   sum on the path has a fixed order).
  *   v, z, norm_w, S_in, m_in, y, S_out, m_out as in ramnet_scan_forward.
  * Errors: as ramnet_scan_forward.
  */
@@ -188,8 +225,10 @@ ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, 
  *              with a message giving both numbers.  Nothing in the array has to start at
  *              zero: each call writes all the scratch it later reads.
  *   Set-up:    the first call on a device (with that device current) looks up the
- *              array's device address once and keeps it; make that first call before
- *              beginning any stream capture.
+ *              array's device address once and keeps it for the current CUDA context; a
+ *              call made in a new context (after cudaDeviceReset, or after the primary
+ *              context was released and created again) looks it up again.  Make the first
+ *              call in a context before beginning any stream capture.
  *   Sharing:   all calls on a device use the same array.  Calls whose work can overlap
  *              on the device (other streams, other host threads) race on it; issue them
  *              on one stream, or use ramnet_scan_forward with separate workspaces.

@@ -75,6 +75,20 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit)
     if (status) atomicOr(status, bit);
 }
 
+// Range check of an index computed on the device.  In a build with RAMNET_DEBUG defined a
+// failing check records kDevCheck in the status word and the caller skips the access; in
+// the normal build the check compiles away.  No trap and no assert either way.
+__device__ __forceinline__ bool dcheck(bool ok, uint32_t* status)
+{
+#ifdef RAMNET_DEBUG
+    if (!ok) set_status(status, kDevCheck);
+    return ok;
+#else
+    (void)status;
+    return ok || true;
+#endif
+}
+
 // ------------------------------------------------------------------ cluster / mbarrier
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -92,15 +106,10 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank)
     return out;
 }
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t caddr)
-{
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
-    return v;
-}
-
-// Whole-cluster hardware barrier; used only right after launch (mbarrier init), where
-// every CTA of the cluster is resident by construction and reaches it unconditionally.
+// Whole-cluster hardware barrier with release/acquire ordering.  Used where every thread of
+// every CTA of the cluster reaches it unconditionally: after the mbarriers are initialised
+// (before any CTA arrives on a peer's barrier) and before exit (so that no CTA leaves while
+// a peer may still write into its shared memory).
 __device__ __forceinline__ void cluster_sync_all()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -116,32 +125,18 @@ __device__ __forceinline__ void fence_mbar_init_cluster()
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// Arrive (release, cluster scope) on the mbarrier at shared::cluster address `caddr`.
+// Arrive (release, cluster scope) on the mbarrier at shared::cluster address `caddr`, which
+// may be in this CTA or in a peer of its cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
 
-// One poll of phase `parity` with acquire at cluster scope.  True once that phase is complete.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity)
+// 16-byte store into a peer CTA's shared memory (shared::cluster address).
+__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d)
 {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait; returns false (and the caller records a timeout) if the phase never completes.
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity)
-{
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-    return false;
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
 // ------------------------------------------------------------------ tensor memory (TMEM)

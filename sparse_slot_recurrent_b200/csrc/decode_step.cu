@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
             const void* lg = stream == 0 ? p.k_logits : p.q_logits;
             const size_t off = static_cast<size_t>(bh) * L;
             uint64_t out[KMAX];
-            if constexpr (KMAX <= 16)
+            if constexpr (KMAX <= 32)
                 topk_search_net<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, out);  // kept list in registers
             else
                 topk_search<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, &kept_s[0][lane], 32, out);
@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
                 if (j < K) {
                     int32_t idx = packed_index(out[j], M);
                     if (cape) idx = cape_shift(idx, pos, M);
+                    if (!dcheck(idx >= 0 && idx < M, p.status)) idx = 0;
                     if (stream == 0) {
                         wi_s[ul][j] = idx;
                         ww_s[ul][j] = w[j];

@@ -80,22 +80,6 @@ uint32_t* device_status_ptr()
     return static_cast<uint32_t*>(p);
 }
 
-// Scratch of the prefill scan: the decoded events [B,H,T,2,K] (16 bytes each), then the
-// fp32 read accumulator [B,T,H,d_v] at a 256-byte boundary.
-struct WorkspaceLayout {
-    size_t o_off, o_bytes, total;
-};
-
-WorkspaceLayout workspace_layout(int B, int T, int H, int K, int d_v, const ramnet::ScanPlan&)
-{
-    WorkspaceLayout w;
-    const size_t events = static_cast<size_t>(B) * H * T * 2 * K * 16;
-    w.o_off = (events + 255) & ~static_cast<size_t>(255);
-    w.o_bytes = static_cast<size_t>(B) * T * H * d_v * sizeof(float);
-    w.total = w.o_off + w.o_bytes;
-    return w;
-}
-
 }  // namespace
 
 namespace ramnet {
@@ -114,8 +98,8 @@ extern "C" {
 const char* ramnet_last_error(void) { return g_last_error.c_str(); }
 
 ramnet_status ramnet_decode_addresses(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, const void* logits,
-                                      ramnet_dtype dt, const int32_t* pos0, const uint8_t* cape_mask,
-                                      int32_t* idx_out, float* w_out, void* stream)
+                                      ramnet_dtype dt, const ramnet_strides* strides, const int32_t* pos0,
+                                      const uint8_t* cape_mask, int32_t* idx_out, float* w_out, void* stream)
 {
     g_last_error.clear();
     int M = 0;
@@ -123,13 +107,29 @@ ramnet_status ramnet_decode_addresses(const ramnet_config* cfg, int32_t B, int32
     if (st != RAMNET_OK) return st;
     if ((st = check_sizes(B, T, H)) != RAMNET_OK) return st;
     if (!valid_dtype(dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype %d", static_cast<int>(dt));
-    REQUIRE_PTR(logits);
+    if (logits == nullptr) return fail(RAMNET_ERR_INVALID_ARG, "logits is NULL");
+    const size_t es = dt == RAMNET_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(logits) & (es - 1)) != 0)
+        return fail(RAMNET_ERR_INVALID_ARG, "logits not aligned to its element size");
+    const int64_t L = static_cast<int64_t>(cfg->U) * cfg->d_p;
+    int64_t sb = static_cast<int64_t>(T) * H * L, stt = static_cast<int64_t>(H) * L, sh = L;
+    if (strides != nullptr) {
+        sb = strides->b;
+        stt = strides->t;
+        sh = strides->h;
+        if (sb < 0 || stt < 0 || sh < 0) return fail(RAMNET_ERR_INVALID_ARG, "negative logits stride");
+        const double span = static_cast<double>(B - 1) * sb + static_cast<double>(T - 1) * stt +
+                            static_cast<double>(H - 1) * sh + static_cast<double>(L);
+        if (span > 9.0e18) return fail(RAMNET_ERR_INVALID_ARG, "logits strides overflow");
+    }
     REQUIRE_PTR(idx_out);
     REQUIRE_PTR(w_out);
     OPTIONAL_PTR(pos0);
     OPTIONAL_PTR(cape_mask);
-    ramnet::DecodeParams p{logits, dt == RAMNET_BF16, cfg->d_p, cfg->U, cfg->K, M, cfg->renorm != 0, B, T, H,
-                           pos0, cape_mask, idx_out, w_out};
+    uint32_t* status = device_status_ptr();
+    if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+    ramnet::DecodeParams p{logits, sb, stt, sh, dt == RAMNET_BF16, cfg->d_p, cfg->U, cfg->K, M, cfg->renorm != 0,
+                           B, T, H, pos0, cape_mask, idx_out, w_out, status};
     cudaError_t e = ramnet::launch_decode_addresses(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode_addresses launch");
     return RAMNET_OK;
@@ -144,10 +144,31 @@ size_t ramnet_scan_workspace_bytes(const ramnet_config* cfg, int32_t B, int32_t 
     for (int in_bytes : {2, 4}) {
         ramnet::ScanPlan plan;
         if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_bytes, &plan)) return 0;
-        const size_t t = workspace_layout(B, T, H, cfg->K, cfg->d_v, plan).total;
+        const size_t t = ramnet::scan_workspace(B, T, H, cfg->K, plan).total;
         total = t > total ? t : total;
     }
     return total;
+}
+
+ramnet_status ramnet_scan_layout(const ramnet_config* cfg, ramnet_dtype in_dt, int32_t* chunk, int32_t* ncta,
+                                 int32_t* scan_warps, int32_t* hdr_words)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet_status st = check_config(cfg, &M);
+    if (st != RAMNET_OK) return st;
+    if (!valid_dtype(in_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype %d", static_cast<int>(in_dt));
+    if (chunk == nullptr || ncta == nullptr || scan_warps == nullptr || hdr_words == nullptr)
+        return fail(RAMNET_ERR_INVALID_ARG, "output pointer is NULL");
+    ramnet::ScanPlan plan;
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, &plan))
+        return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", M,
+                    cfg->d_v);
+    *chunk = plan.chunk;
+    *ncta = plan.ncta;
+    *scan_warps = plan.nw;
+    *hdr_words = plan.hdr_words;
+    return RAMNET_OK;
 }
 
 }  // extern "C"
@@ -158,7 +179,7 @@ namespace {
 // workspace layout.
 ramnet_status check_scan(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
                          const void* workspace, size_t workspace_bytes, int* M, ramnet::ScanPlan* plan,
-                         WorkspaceLayout* wl)
+                         ramnet::ScanWorkspace* wl)
 {
     ramnet_status st = check_config(cfg, M);
     if (st != RAMNET_OK) return st;
@@ -168,18 +189,18 @@ ramnet_status check_scan(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     if (!ramnet::scan_plan(*M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, plan))
         return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", *M,
                     cfg->d_v);
-    *wl = workspace_layout(B, T, H, cfg->K, cfg->d_v, *plan);
+    *wl = ramnet::scan_workspace(B, T, H, cfg->K, *plan);
     if (workspace_bytes < wl->total)
         return fail(RAMNET_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, wl->total);
     return RAMNET_OK;
 }
 
 ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt, int M,
-                         const ramnet::ScanPlan& plan, const WorkspaceLayout& wl, const void* k_logits,
+                         const ramnet::ScanPlan& plan, const ramnet::ScanWorkspace& wl, const void* k_logits,
                          const void* q_logits, const void* g, const uint8_t* cape_mask, const int32_t* pos0,
                          void* workspace, cudaStream_t s)
 {
-    ramnet::EventParams rp{};
+    ramnet::RouteParams rp{};
     rp.k_logits = k_logits;
     rp.q_logits = q_logits;
     rp.g = g;
@@ -194,17 +215,22 @@ ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     rp.H = H;
     rp.pos0 = pos0;
     rp.cape_mask = cape_mask;
+    rp.ncta = plan.ncta;
+    rp.nw = plan.nw;
+    rp.chunk = plan.chunk;
+    rp.nch = (T + plan.chunk - 1) / plan.chunk;
+    rp.hdr_words = plan.hdr_words;
     rp.events = static_cast<uint4*>(workspace);
-    // the read accumulator of the recurrence starts at zero
-    cudaError_t e = cudaMemsetAsync(static_cast<unsigned char*>(workspace) + wl.o_off, 0, wl.o_bytes, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan: accumulator reset");
-    e = ramnet::launch_decode_events(rp, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan: event decode launch");
+    rp.hdr = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(workspace) + wl.hdr_off);
+    rp.status = device_status_ptr();
+    if (rp.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+    cudaError_t e = ramnet::launch_route(rp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan: route launch");
     return RAMNET_OK;
 }
 
 ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt, int M,
-                         const ramnet::ScanPlan& plan, const WorkspaceLayout& wl, const void* v, const void* z,
+                         const ramnet::ScanPlan& plan, const ramnet::ScanWorkspace& wl, const void* v, const void* z,
                          const float* norm_w, const float* S_in, const float* m_in, void* y, ramnet_dtype out_dt,
                          float* S_out, float* m_out, void* workspace, cudaStream_t s)
 {
@@ -212,6 +238,7 @@ ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     if (status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
     ramnet::ScanParams sp{};
     sp.events = static_cast<const uint4*>(workspace);
+    sp.hdr = reinterpret_cast<const uint32_t*>(static_cast<const unsigned char*>(workspace) + wl.hdr_off);
     sp.v = v;
     sp.z = z;
     sp.in_bf16 = in_dt == RAMNET_BF16;
@@ -229,12 +256,18 @@ ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     sp.M = M;
     sp.d_v = cfg->d_v;
     sp.ncta = plan.ncta;
+    sp.nw = plan.nw;
+    sp.nfin = plan.nfin;
     sp.chunk = plan.chunk;
+    sp.nch = (T + plan.chunk - 1) / plan.chunk;
+    sp.stages = plan.stages;
+    sp.lslots = plan.lslots;
+    sp.xslots = plan.xslots;
+    sp.hdr_words = plan.hdr_words;
     sp.eps_gsu = cfg->eps_gsu;
     sp.eps_norm = cfg->eps_norm;
     sp.tmem_cols = plan.tmem_cols;
     sp.status = status;
-    sp.o = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + wl.o_off);
     cudaError_t e = ramnet::launch_scan(sp, plan.smem_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return RAMNET_OK;
@@ -253,7 +286,7 @@ ramnet_status ramnet_scan_forward(const ramnet_config* cfg, int32_t B, int32_t T
     g_last_error.clear();
     int M = 0;
     ramnet::ScanPlan plan;
-    WorkspaceLayout wl;
+    ramnet::ScanWorkspace wl;
     ramnet_status st = check_scan(cfg, B, T, H, in_dt, workspace, workspace_bytes, &M, &plan, &wl);
     if (st != RAMNET_OK) return st;
     if (!valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
@@ -284,7 +317,7 @@ ramnet_status ramnet_scan_route(const ramnet_config* cfg, int32_t B, int32_t T, 
     g_last_error.clear();
     int M = 0;
     ramnet::ScanPlan plan;
-    WorkspaceLayout wl;
+    ramnet::ScanWorkspace wl;
     ramnet_status st = check_scan(cfg, B, T, H, in_dt, workspace, workspace_bytes, &M, &plan, &wl);
     if (st != RAMNET_OK) return st;
     REQUIRE_PTR(k_logits);
@@ -304,7 +337,7 @@ ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, 
     g_last_error.clear();
     int M = 0;
     ramnet::ScanPlan plan;
-    WorkspaceLayout wl;
+    ramnet::ScanWorkspace wl;
     ramnet_status st = check_scan(cfg, B, T, H, in_dt, workspace, workspace_bytes, &M, &plan, &wl);
     if (st != RAMNET_OK) return st;
     if (!valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
@@ -378,6 +411,8 @@ ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H,
     p.renorm = cfg->renorm != 0;
     p.eps_gsu = cfg->eps_gsu;
     p.eps_norm = cfg->eps_norm;
+    p.status = device_status_ptr();
+    if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
     cudaError_t e = ramnet::launch_decode_step(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
     return RAMNET_OK;

@@ -1,38 +1,39 @@
-// scan_forward.cu -- K2: the prefill recurrence of the RAM-Net layer core, and K2b: the
-// output normalisation.
+// scan_forward.cu -- second launch of the prefill scan: the recurrence of the RAM-Net layer
+// core (Gated Sparse Update, sparse read, RMSNorm, output gate) over the events that the
+// route kernel grouped by owner.
 //
-// RAM-Net project page: the three-stage paragraph (decode, CAPE, GSU, then read,
-// normalise, gate), the Gated Sparse Update paragraphs (four steps; unselected slots
-// unchanged) and the GPU-execution paragraph (addresses for all tokens first, events
-// grouped by slot, each slot's events walked in causal order, slots and channels in
-// parallel).
+// RAM-Net project page: the three-stage paragraph (decode, CAPE, GSU, then read, normalise,
+// gate), the Gated Sparse Update paragraphs (four steps; unselected slots unchanged) and the
+// GPU-execution paragraph (events grouped by slot, each slot's events walked in causal
+// order, slots and channels in parallel, slots without events cost nothing).
 //
 // State layout.  One head's slot array S [M, d_v] fp32 lives in tensor memory (TMEM) for
-// the whole sequence, spread over `ncta` CTAs, one per SM.  Slot i belongs to CTA
-// (i mod ncta) as local slot s = i / ncta, which sits in TMEM lane quadrant (s mod 4),
-// columns [(s/4)*CPL, (s/4)*CPL + CPL); lane l of the quadrant holds channels
-// [l*CPL, l*CPL + CPL).  One slot row is one tcgen05.ld/st of CPL columns by a warp of
-// that quadrant.  Scan warp w (0..15) owns the local slots with s mod 16 == w and walks
-// their events in token order (a token's writes before its reads).
+// the whole sequence, spread over a cluster of `ncta` CTAs, one per SM.  Slot i belongs to
+// CTA rank (i mod ncta) as local slot s = i / ncta, which sits in TMEM lane quadrant
+// (s mod 4), columns [(s/4)*CPL, (s/4)*CPL + CPL); lane l of the quadrant holds channels
+// [l*CPL, l*CPL + CPL).  One slot row is one tcgen05.ld/st of CPL columns by a warp of that
+// quadrant.  Scan warp w owns the local slots with s mod nw == w.
 //
-// Per CTA: a loader warp bulk-copies each chunk's events (C tokens, token order, as the
-// event decode wrote them) and value rows into a ring of kStages shared-memory stages;
-// each scan warp picks its own events out of the chunk 32 at a time (one ballot per 32
-// events) and walks them at its own pace (no barrier between scan warps; a stage is
-// recycled once all 16 have left it):
-//   write event  GSU steps 1-3 on the slot's mass (m = alpha*m + w, lambda = w/(m+eps),
-//                m kept in shared memory), step 4 on the row (tcgen05.ld, update,
-//                tcgen05.st);
-//   read event   the weighted row r*S is added into the token's read accumulator o
-//                [B,T,H,d_v] fp32 in global memory (vector red.add), which
-//                ramnet_scan_route reset to zero.  The read of token t follows t's own
-//                writes in the list.
-// K2b then turns o into y: RMSNorm over d_v, norm weight, output gate.  The read
-// accumulator adds up to K terms per element in an order that can change from run to
-// run, so y may differ between runs in the last bits.
+// Warps of a CTA:
+//   loader      bulk-copies each chunk's header, this CTA's events and the chunk's value
+//               rows into a ring of `stages` shared-memory stages;
+//   scan warps  each walks its own event list of the chunk (token order, a token's writes
+//               before its reads) in batches of up to kBatch events on distinct slots: one
+//               tcgen05.ld per event, one wait per batch (a TMEM load takes a few hundred
+//               cycles), then per write GSU steps 1-4 (mass m = alpha*m + w, rate
+//               lambda = w/(m + eps), row S <- S + lambda (v - S), stored back with
+//               tcgen05.st) and per read the weighted row r*S, stored into this CTA's
+//               read-partial ring at (token, q), q = the read's rank among the token's
+//               reads held by this CTA;
+//   finishers   per token, the sum of the CTA's read partials in q order; the CTA that
+//               finishes the chunk (rank = chunk mod ncta) adds the peers' sums in rank
+//               order (peers store theirs into its shared memory: one row per token), then
+//               RMSNorm over d_v, norm weight, output gate, y.
+// Every sum has a fixed order, so y is the same from run to run.
 // Every wait is bounded (about 2 s); a wait that gives up records RAMNET_ERR_TIMEOUT in the
-// status word, raises the CTA's abort flag and the kernel carries on to the end without
-// further waiting (all loops are bounded by the chunk's event capacity).
+// status word and raises the CTA's abort flag, after which its waits return at once, scan
+// warps skip their events and the loader stops copying, so the kernel ends within seconds.
+// Event fields are checked against their ranges before use (RAMNET_ERR_DEVICE_CHECK).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -40,41 +41,62 @@ namespace ramnet {
 
 namespace {
 
-constexpr int kScanWarps = 16;
-constexpr int kThreads = (kScanWarps + 1) * 32;
-constexpr int kStages = 8;  // staging ring depth: a scan warp may run up to 7 chunks ahead
-
-// mbarrier indices
-constexpr int kBarStage = 0;                        // [kStages] staged data landed (tx)
-constexpr int kBarFree = kBarStage + kStages;       // [kStages] every scan warp left the stage
-constexpr int kNumBars = kBarFree + kStages;
+constexpr int kBatch = 8;  // events per TMEM round trip of a scan warp
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
+// mbarrier indices
+struct Bars {
+    int sfull, sfree, ldone, lfree, xfull, xfree, count;
+};
+__host__ __device__ inline Bars bar_index(int S, int P, int X, int ncta)
+{
+    Bars b;
+    b.sfull = 0;            // [S] stage landed (loader arrive + bulk-copy bytes)
+    b.sfree = S;            // [S] every scan warp left the stage
+    b.ldone = 2 * S;        // [P] every scan warp stored its read partials of the chunk
+    b.lfree = 2 * S + P;    // [P] the finishers summed the chunk's partials
+    b.xfull = 2 * S + 2 * P;          // [X] every peer stored its sums of a chunk this CTA finishes
+    b.xfree = 2 * S + 2 * P + X;      // [ncta][X] finisher CTA f released its exchange slot
+    b.count = 2 * S + 2 * P + X + ncta * X;
+    return b;
+}
+
 struct Layout {
-    size_t bars, misc, m, stage, total;
-    size_t stage_bytes, v_off;
+    size_t bars, misc, m, nloc, stage, stage_bytes, ev_off, v_off, lring, lring_bytes, xbuf, xbuf_bytes, total;
 };
 
-// Shared memory of the scan kernel: barriers, masses of the CTA's slots, and kStages stages
-// of [C tokens x 2 streams x K events] 16-byte records followed by C value rows.
-__host__ __device__ inline Layout scan_layout(int Ml, int C, int K, int dv, int es)
+// Shared memory of the scan kernel.
+__host__ __device__ inline Layout scan_layout(int Ml, int C, int K, int dv, int es, int S, int P, int X, int ncta,
+                                              int hw)
 {
     Layout L;
-    L.v_off = static_cast<size_t>(C) * 2 * K * sizeof(uint4);
-    L.stage_bytes = L.v_off + align16(static_cast<size_t>(C) * dv * es);
+    const Bars b = bar_index(S, P, X, ncta);
     size_t o = 0;
     L.bars = o;
-    o += align16(8 * kNumBars);
+    o += align16(8 * static_cast<size_t>(b.count));
     L.misc = o;
     o += 16;
     L.m = o;
     o += align16(sizeof(float) * Ml);
+    L.nloc = o;
+    o += align16(static_cast<size_t>(P) * C);
+    L.ev_off = align16(static_cast<size_t>(hw) * 4);
+    L.v_off = L.ev_off + static_cast<size_t>(C) * 2 * K * sizeof(uint4);
+    L.stage_bytes = L.v_off + align16(static_cast<size_t>(C) * dv * es);
     L.stage = o;
-    o += kStages * L.stage_bytes;
+    o += static_cast<size_t>(S) * L.stage_bytes;
+    L.lring_bytes = static_cast<size_t>(C) * K * dv * sizeof(float);
+    L.lring = o;
+    o += static_cast<size_t>(P) * L.lring_bytes;
+    L.xbuf_bytes = static_cast<size_t>(ncta > 1 ? ncta - 1 : 0) * C * dv * sizeof(float);
+    L.xbuf = o;
+    o += static_cast<size_t>(X) * L.xbuf_bytes;
     L.total = o;
     return L;
 }
+
+__host__ __device__ inline int hdr_words_of(int nw, int C) { return (4 + nw + 1 + (C + 3) / 4 + 3) & ~3; }
 
 __device__ __forceinline__ uint64_t global_ns()
 {
@@ -83,8 +105,8 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// One try_wait on phase `parity`: the thread is suspended in hardware until the phase
-// completes or about kSuspendNs have passed, so a waiting warp issues almost nothing.
+// One try_wait on phase `parity` (acquire at cluster scope): the thread is suspended in
+// hardware until the phase completes or about kSuspendNs have passed.
 constexpr uint32_t kSuspendNs = 100000;
 
 __device__ __forceinline__ bool try_wait_cta(uint32_t bar, uint32_t parity)
@@ -92,7 +114,7 @@ __device__ __forceinline__ bool try_wait_cta(uint32_t bar, uint32_t parity)
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity), "r"(kSuspendNs)
@@ -128,11 +150,6 @@ __device__ __noinline__ void drain_copies(uint32_t bar, uint32_t parity)
     }
 }
 
-__device__ __forceinline__ void arrive_cta(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
 __device__ __forceinline__ void arrive_expect_tx(uint32_t bar, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -147,6 +164,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Named barrier of the finisher warps (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void finisher_sync(int nthreads)
+{
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
 
 // CPL consecutive input elements (fp32 or bf16) from shared memory, as fp32.
 template <int CPL>
@@ -185,15 +208,53 @@ __device__ __forceinline__ void load_row(const unsigned char* base, int elem, in
     }
 }
 
+// CPL consecutive elements of a global [.., d_v] input row as fp32.
 template <int CPL>
-__device__ __forceinline__ void store_row(float* dst, const float (&v)[CPL])
+__device__ __forceinline__ void load_row_in(const void* base, size_t elem, int is_bf16, float (&v)[CPL])
+{
+    if (is_bf16) {
+        const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(base) + elem;
+        if constexpr (CPL % 4 == 0) {
+#pragma unroll
+            for (int c = 0; c < CPL; c += 4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(pb + c);
+                v[c + 0] = __uint_as_float(u.x << 16);
+                v[c + 1] = __uint_as_float(u.x & 0xFFFF0000u);
+                v[c + 2] = __uint_as_float(u.y << 16);
+                v[c + 3] = __uint_as_float(u.y & 0xFFFF0000u);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) v[c] = __bfloat162float(pb[c]);
+        }
+    } else {
+        load_row_g<CPL>(reinterpret_cast<const float*>(base) + elem, v);
+    }
+}
+
+template <int CPL>
+__device__ __forceinline__ void lds_row(const float* p, float (&v)[CPL])
+{
+    load_row_g<CPL>(p, v);  // generic vector loads of shared memory
+}
+
+template <int CPL>
+__device__ __forceinline__ void sts_row(float* p, const float (&v)[CPL])
+{
+    store_row_g<CPL>(p, v);
+}
+
+// CPL values into a peer CTA's shared memory at shared::cluster address `caddr`.
+template <int CPL>
+__device__ __forceinline__ void st_cluster_row(uint32_t caddr, const float (&v)[CPL])
 {
     if constexpr (CPL % 4 == 0) {
 #pragma unroll
-        for (int c = 0; c < CPL; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+        for (int c = 0; c < CPL; c += 4) st_cluster_v4(caddr + 4 * c, v[c], v[c + 1], v[c + 2], v[c + 3]);
     } else {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) dst[c] = v[c];
+        for (int c = 0; c < CPL; ++c)
+            asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr + 4 * c), "f"(v[c]) : "memory");
     }
 }
 
@@ -218,79 +279,74 @@ __device__ __forceinline__ void store_y(void* y, size_t elem, const float (&v)[C
             for (int c = 0; c < CPL; ++c) pb[c] = __float2bfloat16_rn(v[c]);
         }
     } else {
-        float* pf = reinterpret_cast<float*>(y) + elem;
-        if constexpr (CPL % 4 == 0) {
-#pragma unroll
-            for (int c = 0; c < CPL; c += 4) *reinterpret_cast<float4*>(pf + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-        } else {
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) pf[c] = v[c];
-        }
+        store_row_g<CPL>(reinterpret_cast<float*>(y) + elem, v);
     }
 }
 
-// o[0..CPL) += v[0..CPL) in global memory, vector reductions (p 4*CPL-byte aligned).
-template <int CPL>
-__device__ __forceinline__ void red_add_row(float* p, const float (&v)[CPL])
-{
-    if constexpr (CPL == 1) {
-        asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v[0]) : "memory");
-    } else if constexpr (CPL == 2) {
-        asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v[0]), "f"(v[1]) : "memory");
-    } else {
-#pragma unroll
-        for (int c = 0; c < CPL; c += 4)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p + c), "f"(v[c]), "f"(v[c + 1]),
-                         "f"(v[c + 2]), "f"(v[c + 3])
-                         : "memory");
-    }
-}
+constexpr int kScanWarps = 16;
+constexpr int kFinWarps = 8;
+constexpr int kScanThreads = (kScanWarps + kFinWarps + 1) * 32;
+constexpr int kSmemBudget = 220 * 1024;
 
 template <int CPL>
-__global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
+__global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int C = p.chunk, dv = p.d_v, ncta = p.ncta, M = p.M, K = p.K;
+    constexpr int kZMax = 8;  // z values a finisher lane prefetches per chunk
+    const int C = p.chunk, dv = p.d_v, ncta = p.ncta, M = p.M, K = p.K, NW = p.nw, F = p.nfin;
+    const int S = p.stages, P = p.lslots, X = p.xslots;
     const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;  // lanes holding channels (32 unless d_v = 16)
     const int es = p.in_bf16 ? 2 : 4;
-    const int rank = static_cast<int>(blockIdx.x) % ncta;
+    const int rank = static_cast<int>(cluster_ctarank());
     const int bh = static_cast<int>(blockIdx.x) / ncta;
     const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Ml = (M - rank + ncta - 1) / ncta;
-    const int nch = (p.T + C - 1) / C;
-    const int lg_ncta = __ffs(ncta) - 1;
-    const Layout L = scan_layout((M + ncta - 1) / ncta, C, K, dv, es);
+    const int nch = p.nch;
+    const int cap = 2 * C * K;  // event capacity of a stage
+    const Layout L = scan_layout((M + ncta - 1) / ncta, C, K, dv, es, S, P, X, ncta, p.hdr_words);
+    const Bars BI = bar_index(S, P, X, ncta);
     const uint32_t bars = smem_addr(smem + L.bars);
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
     uint64_t* bar_ptr = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint32_t* holder = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
     float* m_s = reinterpret_cast<float*>(smem + L.m);
-    auto stage = [&](int c) { return smem + L.stage + static_cast<size_t>(c % kStages) * L.stage_bytes; };
+    unsigned char* nloc_s = smem + L.nloc;
+    auto stage = [&](int c) { return smem + L.stage + static_cast<size_t>(c % S) * L.stage_bytes; };
+    float* lring = reinterpret_cast<float*>(smem + L.lring);
+    const size_t lslot_floats = L.lring_bytes / sizeof(float);
+    float* xbuf = reinterpret_cast<float*>(smem + L.xbuf);
+    const size_t xslot_floats = L.xbuf_bytes / sizeof(float);
 
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(bar_ptr + kBarStage + i, 1);
-            mbar_init(bar_ptr + kBarFree + i, kScanWarps * 32);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(bar_ptr + BI.sfull + i, 1);
+            mbar_init(bar_ptr + BI.sfree + i, NW);
         }
+        for (int i = 0; i < P; ++i) {
+            mbar_init(bar_ptr + BI.ldone + i, NW);
+            mbar_init(bar_ptr + BI.lfree + i, 1);
+        }
+        for (int i = 0; i < X; ++i) mbar_init(bar_ptr + BI.xfull + i, ncta > 1 ? ncta - 1 : 1);
+        for (int i = 0; i < ncta * X; ++i) mbar_init(bar_ptr + BI.xfree + i, 1);
         fence_mbar_init_cluster();
     }
     if (warp == 0) tmem_alloc(holder, p.tmem_cols);
-    for (int s = tid; s < Ml; s += kThreads)
+    for (int s = tid; s < Ml; s += blockDim.x)
         m_s[s] = p.m_in != nullptr ? p.m_in[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] : 0.0f;
     tmem_fence_before_sync();
-    __syncthreads();
+    cluster_sync_all();  // barriers initialised cluster-wide before any peer arrives on them
     tmem_fence_after_sync();
     const uint32_t tbase = *holder;
 
-    if (warp < kScanWarps) {
+    if (warp < NW) {
         // ============================================================ scan warps
-        const int q = warp & 3;
-        const uint32_t tq = tbase + (static_cast<uint32_t>(32 * q) << 16);
+        const int q4 = warp & 3;
+        const uint32_t tq = tbase + (static_cast<uint32_t>(32 * q4) << 16);
         const int lch = (lane < LW ? lane : 0) * CPL;  // this lane's first channel
-        for (int s = warp; s < Ml; s += kScanWarps) {
+        for (int s = warp; s < Ml; s += NW) {
             const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
             float r[CPL];
 #pragma unroll
@@ -298,60 +354,99 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             tmem_st<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), r);
         }
         tmem_wait_st();
+        const unsigned lt_mask = (1u << lane) - 1u;
         for (int c = 0; c < nch; ++c) {
-            wait_bounded(bar(kBarStage + c % kStages), (c / kStages) & 1, p.status, abort_flag);
+            wait_bounded(bar(BI.sfull + c % S), (c / S) & 1, p.status, abort_flag);
+            const int ls = c % P, kl = c / P;
+            if (kl >= 1) wait_bounded(bar(BI.lfree + ls), (kl - 1) & 1, p.status, abort_flag);
             const unsigned char* st = stage(c);
-            const uint4* evs = reinterpret_cast<const uint4*>(st);
-            const unsigned char* vb = st + L.v_off;
-            const int nev = min(C, p.T - c * C) * 2 * K;
-            const int t0 = c * C;
-            // o row of token t0 of this chunk; token t at + (t - t0) * H * d_v
-            float* orow0 = p.o + ((static_cast<size_t>(b) * p.T + t0) * p.H + h) * dv + lch;
-            const size_t ostride = static_cast<size_t>(p.H) * dv;
-            uint4 rn = lane < nev ? evs[lane] : make_uint4(0u, 0u, 0u, 0u);  // next group, prefetched
-            for (int base = 0; base < nev; base += 32) {
-                const int e = base + lane;
-                const uint4 r = rn;
-                if (base + 32 < nev) rn = e + 32 < nev ? evs[e + 32] : make_uint4(0u, 0u, 0u, 0u);
-                const int sloc = static_cast<int>(r.x >> lg_ncta);
-                const bool mine = e < nev && static_cast<int>(r.x & (ncta - 1)) == rank && (sloc & (kScanWarps - 1)) == warp;
-                uint32_t mask = __ballot_sync(0xffffffffu, mine);
-                while (mask != 0u) {
-                    const int src = __ffs(mask) - 1;
-                    mask &= mask - 1u;
-                    const int sl = __shfl_sync(0xffffffffu, sloc, src);
-                    const float cf = __uint_as_float(__shfl_sync(0xffffffffu, r.y, src));
-                    const float al = __uint_as_float(__shfl_sync(0xffffffffu, r.z, src));
-                    const uint32_t tag = __shfl_sync(0xffffffffu, r.w, src);
-                    const int tl = static_cast<int>(tag >> 1) - t0;
-                    const uint32_t col = static_cast<uint32_t>((sl >> 2) * CPL);
-                    float S[CPL];
-                    tmem_ld<CPL>(tq + col, S);
-                    if ((tag & 1u) == 0u) {
-                        // write: GSU steps 1-3, m = alpha*m + w, lambda = w / (m + eps); step 4
-                        float vv[CPL];
-                        load_row<CPL>(vb, tl * dv + lch, p.in_bf16, vv);
-                        const float mn = fmaf(al, m_s[sl], cf);
-                        const float lam = __fdividef(cf, mn + p.eps_gsu);
-                        m_s[sl] = mn;  // every lane stores the same value and later reads its own store
-                        tmem_wait_ld();
+            const uint32_t* hd = reinterpret_cast<const uint32_t*>(st);
+            if (!*abort_flag) {
+                const int nt = min(static_cast<int>(hd[2]), C);
+                const int beg = min(static_cast<int>(hd[4 + warp]), cap);
+                const int end = max(beg, min(static_cast<int>(hd[5 + warp]), cap));
+                if (warp == 0) {
+                    const unsigned char* nb = st + (4 + NW + 1) * 4;
+                    for (int i = lane; i < C; i += 32) nloc_s[ls * C + i] = nb[i];
+                }
+                const uint4* evs = reinterpret_cast<const uint4*>(st + L.ev_off);
+                const unsigned char* vb = st + L.v_off;
+                float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
+                int e = beg;
+                while (e < end) {
+                    // the longest run of up to kBatch events on distinct slots
+                    const int navail = end - e;
+                    uint32_t sl = 0x10000u + static_cast<uint32_t>(lane);
+                    if (lane < kBatch && lane < navail) sl = evs[e + lane].x & 0xFFFFu;
+                    const uint32_t peers = __match_any_sync(0xffffffffu, sl);
+                    const uint32_t dup = __ballot_sync(0xffffffffu, (peers & lt_mask) != 0u);
+                    int nb = min(navail, kBatch);
+                    if (dup != 0u) nb = min(nb, __ffs(dup) - 1);
+                    uint32_t xk[kBatch];
+                    float ck[kBatch];
+                    float Sv[kBatch][CPL];
 #pragma unroll
-                        for (int cc = 0; cc < CPL; ++cc) S[cc] = fmaf(lam, vv[cc] - S[cc], S[cc]);
-                        tmem_st<CPL>(tq + col, S);
-                        tmem_wait_st();
-                    } else {
-                        // read: r * S into the token's read accumulator
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int cc = 0; cc < CPL; ++cc) S[cc] *= cf;
-                        if (lane < LW) red_add_row<CPL>(orow0 + static_cast<size_t>(tl) * ostride, S);
+                    for (int k = 0; k < kBatch; ++k) {
+                        xk[k] = 0xFFFFFFFFu;
+                        if (k < nb) {
+                            const uint4 r = evs[e + k];
+                            const int s = static_cast<int>(r.x & 0xFFFFu);
+                            const int tl = static_cast<int>((r.x >> 16) & 0xFFu);
+                            const bool rd = (r.x >> 31) != 0u;
+                            const int q = static_cast<int>((r.x >> 24) & 0x3Fu);
+                            if (s < Ml && (s & (NW - 1)) == warp && tl < nt && (!rd || q < K)) {
+                                xk[k] = r.x;
+                                tmem_ld<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), Sv[k]);
+                                const float w = __uint_as_float(r.y);
+                                if (!rd) {
+                                    // GSU steps 1-3: m = alpha*m + w, lambda = w / (m + eps)
+                                    const float mn = fmaf(__uint_as_float(r.z), m_s[s], w);
+                                    m_s[s] = mn;  // every lane stores the same value
+                                    ck[k] = __fdividef(w, mn + p.eps_gsu);
+                                } else {
+                                    ck[k] = w;
+                                }
+                            } else {
+                                set_status(p.status, kDevCheck);
+                            }
+                        }
                     }
+                    tmem_wait_ld();
+                    bool wrote = false;
+#pragma unroll
+                    for (int k = 0; k < kBatch; ++k) {
+                        if (k < nb && xk[k] != 0xFFFFFFFFu) {
+                            const int s = static_cast<int>(xk[k] & 0xFFFFu);
+                            const int tl = static_cast<int>((xk[k] >> 16) & 0xFFu);
+                            if ((xk[k] >> 31) == 0u) {
+                                // GSU step 4 on the row
+                                float vv[CPL];
+                                load_row<CPL>(vb, tl * dv + lch, p.in_bf16, vv);
+#pragma unroll
+                                for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] = fmaf(ck[k], vv[cc] - Sv[k][cc], Sv[k][cc]);
+                                tmem_st<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), Sv[k]);
+                                wrote = true;
+                            } else {
+                                // read: r * S into the partial ring at (token, q)
+                                const int q = static_cast<int>((xk[k] >> 24) & 0x3Fu);
+#pragma unroll
+                                for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] *= ck[k];
+                                if (lane < LW) sts_row<CPL>(lr + static_cast<size_t>(tl * K + q) * dv, Sv[k]);
+                            }
+                        }
+                    }
+                    if (wrote) tmem_wait_st();
+                    e += nb;
                 }
             }
-            arrive_cta(bar(kBarFree + c % kStages));
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_cluster(map_to_rank(bar(BI.sfree + c % S), static_cast<uint32_t>(rank)));
+                mbar_arrive_cluster(map_to_rank(bar(BI.ldone + ls), static_cast<uint32_t>(rank)));
+            }
         }
         // final state of the owned slots
-        for (int s = warp; s < Ml; s += kScanWarps) {
+        for (int s = warp; s < Ml; s += NW) {
             const size_t row = (static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank) * dv;
             float r[CPL];
             tmem_ld<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), r);
@@ -362,68 +457,166 @@ __global__ void __launch_bounds__(kThreads, 1) k_scan(ScanParams p)
             }
             if (lane == 0) p.m_out[static_cast<size_t>(bh) * M + static_cast<size_t>(s) * ncta + rank] = m_s[s];
         }
+    } else if (warp < NW + F) {
+        // ============================================================ finisher warps
+        const int fw = warp - NW;
+        const int lch = (lane < LW ? lane : 0) * CPL;
+        float nwv[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) nwv[c] = p.norm_w != nullptr ? p.norm_w[lch + c] : 1.0f;
+        const int ft = (C + F - 1) / F;  // tokens per finisher warp per chunk (ft * CPL <= kZMax)
+        for (int c = 0; c < nch; ++c) {
+            const int ls = c % P, kl = c / P;
+            const int f = c % ncta;
+            const int xs = (c / ncta) % X, kx = c / (ncta * X);
+            const int nt = min(C, p.T - c * C);
+            const bool own = f == rank;
+            const int t0 = c * C;
+            float zr[kZMax];
+#pragma unroll
+            for (int i = 0; i < kZMax; ++i) zr[i] = 0.0f;
+            if (own) {
+#pragma unroll
+                for (int i = 0; i < kZMax / CPL; ++i) {
+                    const int tl = fw + i * F;
+                    if (i < ft && tl < nt && lane < LW) {
+                        float zz[CPL];
+                        load_row_in<CPL>(p.z, ((static_cast<size_t>(b) * p.T + t0 + tl) * p.H + h) * dv + lch, p.in_bf16,
+                                         zz);
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) zr[i * CPL + cc] = zz[cc];
+                    }
+                }
+            }
+            wait_bounded(bar(BI.ldone + ls), kl & 1, p.status, abort_flag);
+            if (ncta > 1) {
+                if (own) wait_bounded(bar(BI.xfull + xs), kx & 1, p.status, abort_flag);
+                else if (kx >= 1) wait_bounded(bar(BI.xfree + f * X + xs), (kx - 1) & 1, p.status, abort_flag);
+            }
+            const float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
+            const int xi = rank < f ? rank : rank - 1;  // this CTA's entry in f's exchange slot
+            const uint32_t xdst = ncta > 1 && !own
+                                      ? map_to_rank(smem_addr(xbuf + static_cast<size_t>(xs) * xslot_floats +
+                                                              static_cast<size_t>(xi) * C * dv + lch),
+                                                    static_cast<uint32_t>(f))
+                                      : 0u;
+#pragma unroll
+            for (int i = 0; i < kZMax / CPL; ++i) {
+                const int tl = fw + i * F;
+                if (i < ft && tl < nt) {
+                    const int n = min(static_cast<int>(nloc_s[ls * C + tl]), K);
+                    float o[CPL];
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) o[cc] = 0.0f;
+                    for (int q = 0; q < n; ++q) {
+                        float pr[CPL];
+                        lds_row<CPL>(lr + static_cast<size_t>(tl * K + q) * dv, pr);
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) o[cc] += pr[cc];
+                    }
+                    if (own) {
+                        // rank order: peers below this CTA, this CTA, peers above
+                        float tot[CPL];
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) tot[cc] = 0.0f;
+                        for (int r2 = 0; r2 < ncta; ++r2) {
+                            if (r2 == rank) {
+#pragma unroll
+                                for (int cc = 0; cc < CPL; ++cc) tot[cc] += o[cc];
+                            } else {
+                                const int xi2 = r2 < rank ? r2 : r2 - 1;
+                                float pr[CPL];
+                                lds_row<CPL>(xbuf + static_cast<size_t>(xs) * xslot_floats +
+                                                 (static_cast<size_t>(xi2) * C + tl) * dv + lch,
+                                             pr);
+#pragma unroll
+                                for (int cc = 0; cc < CPL; ++cc) tot[cc] += pr[cc];
+                            }
+                        }
+                        float ss = 0.0f;
+                        if (lane < LW) {
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) ss = fmaf(tot[cc], tot[cc], ss);
+                        }
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                        const float inv = 1.0f / sqrtf(ss / dv + p.eps_norm);
+                        if (lane < LW && !*abort_flag) {
+                            float yv[CPL];
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) yv[cc] = tot[cc] * inv * nwv[cc] * zr[i * CPL + cc];
+                            store_y<CPL>(p.y, ((static_cast<size_t>(b) * p.T + t0 + tl) * p.H + h) * dv + lch, yv,
+                                         p.out_bf16);
+                        }
+                    } else if (lane < LW) {
+                        st_cluster_row<CPL>(xdst + static_cast<uint32_t>(tl * dv * 4), o);
+                    }
+                }
+            }
+            finisher_sync(F * 32);
+            if (fw == 0 && lane == 0) {
+                mbar_arrive_cluster(map_to_rank(bar(BI.lfree + ls), static_cast<uint32_t>(rank)));
+                if (ncta > 1) {
+                    if (own) {
+                        for (int r2 = 0; r2 < ncta; ++r2)
+                            if (r2 != rank)
+                                mbar_arrive_cluster(map_to_rank(bar(BI.xfree + rank * X + xs), static_cast<uint32_t>(r2)));
+                    } else {
+                        mbar_arrive_cluster(map_to_rank(bar(BI.xfull + xs), static_cast<uint32_t>(f)));
+                    }
+                }
+            }
+        }
     } else {
         // ============================================================ loader warp
         const uint32_t vrow = static_cast<uint32_t>(dv * es);
+        const uint32_t hdr_bytes = static_cast<uint32_t>(p.hdr_words * 4);
+        uint32_t pf_start = 0, pf_n = 0;  // (first event, count) of chunk (c & ~31) + lane
+        int issued = 0;                    // chunks whose copies were issued (0..issued-1)
         for (int c = 0; c < nch; ++c) {
-            const int n = min(C, p.T - c * C);
-            if (c >= kStages) {
-                wait_bounded(bar(kBarFree + c % kStages), (c / kStages - 1) & 1, p.status, abort_flag);
+            if ((c & 31) == 0) {
+                const int cc = c + lane;
+                if (cc < nch) {
+                    const uint32_t* hp = p.hdr + ((static_cast<size_t>(bh) * nch + cc) * ncta + rank) * p.hdr_words;
+                    pf_start = hp[0];
+                    pf_n = hp[1];
+                }
+            }
+            const uint32_t start = __shfl_sync(0xffffffffu, pf_start, c & 31);
+            const uint32_t n = min(__shfl_sync(0xffffffffu, pf_n, c & 31), static_cast<uint32_t>(cap));
+            const uint32_t first = min(start, static_cast<uint32_t>(cap) - n);
+            const int nt = min(C, p.T - c * C);
+            if (c >= S) {
+                wait_bounded(bar(BI.sfree + c % S), (c / S - 1) & 1, p.status, abort_flag);
                 fence_proxy_async();
             }
+            if (*abort_flag) continue;
             unsigned char* st = stage(c);
-            const uint32_t sb = bar(kBarStage + c % kStages);
-            const uint32_t evb = static_cast<uint32_t>(n * 2 * K * sizeof(uint4));
-            if (lane == 0) arrive_expect_tx(sb, evb + static_cast<uint32_t>(n) * vrow);
+            const uint32_t sb = bar(BI.sfull + c % S);
+            const uint32_t evb = n * static_cast<uint32_t>(sizeof(uint4));
+            if (lane == 0) arrive_expect_tx(sb, hdr_bytes + evb + static_cast<uint32_t>(nt) * vrow);
             __syncwarp();
-            if (lane == 0)
-                bulk_g2s(smem_addr(st), p.events + (static_cast<size_t>(bh) * p.T + static_cast<size_t>(c) * C) * 2 * K, evb,
-                         sb);
-            for (int t = lane; t < n; t += 32) {
-                const size_t th = (static_cast<size_t>(b) * p.T + c * C + t) * p.H + h;
+            if (lane == 0) {
+                bulk_g2s(smem_addr(st), p.hdr + ((static_cast<size_t>(bh) * nch + c) * ncta + rank) * p.hdr_words,
+                         hdr_bytes, sb);
+                if (evb > 0)
+                    bulk_g2s(smem_addr(st + L.ev_off),
+                             p.events + (static_cast<size_t>(bh) * nch + c) * static_cast<size_t>(cap) + first, evb, sb);
+            }
+            for (int t = lane; t < nt; t += 32) {
+                const size_t th = (static_cast<size_t>(b) * p.T + static_cast<size_t>(c) * C + t) * p.H + h;
                 bulk_g2s(smem_addr(st + L.v_off + static_cast<size_t>(t) * vrow),
                          static_cast<const unsigned char*>(p.v) + th * vrow, vrow, sb);
             }
+            issued = c + 1;
         }
-        for (int c = max(0, nch - kStages); c < nch; ++c) drain_copies(bar(kBarStage + c % kStages), (c / kStages) & 1);
+        for (int c = max(0, issued - S); c < issued; ++c) drain_copies(bar(BI.sfull + c % S), (c / S) & 1);
     }
 
     tmem_fence_before_sync();
-    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while a peer may still store into its shared memory
     tmem_fence_after_sync();
     if (warp == 0) tmem_dealloc(tbase, p.tmem_cols);
-}
-
-// K2b: y = o / sqrt(mean(o^2) + eps) * norm_w * z for every token-head, one warp each.
-template <int CPL>
-__global__ void __launch_bounds__(256) k_scan_norm(ScanParams p)
-{
-    const int lane = threadIdx.x & 31;
-    const size_t th = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    const size_t n_th = static_cast<size_t>(p.B) * p.T * p.H;
-    if (th >= n_th) return;
-    const int dv = p.d_v;
-    const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;
-    const int lch = (lane < LW ? lane : 0) * CPL;
-    float o[CPL];
-    load_row_g<CPL>(p.o + th * dv + lch, o);
-    float ss = 0.0f;
-    if (lane < LW) {
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) ss = fmaf(o[c], o[c], ss);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float inv = 1.0f / sqrtf(ss / dv + p.eps_norm);
-    if (lane < LW) {
-        float yv[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            const float nw = p.norm_w != nullptr ? p.norm_w[lch + c] : 1.0f;
-            yv[c] = o[c] * inv * nw * load_in(p.z, th * dv + lch + c, p.in_bf16);
-        }
-        store_y<CPL>(p.y, th * dv + lch, yv, p.out_bf16);
-    }
 }
 
 // Failure-detection self-test: one thread waits, through wait_bounded, on a barrier that
@@ -460,40 +653,70 @@ bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
     const int cols = ((Ml + 3) / 4) * cpl;
     uint32_t alloc = 32;
     while (alloc < static_cast<uint32_t>(cols)) alloc <<= 1;
-    auto total = [&](int cc) { return scan_layout(Ml, cc, K, d_v, in_bytes).total; };
-    const size_t budget = 200 * 1024;
+    const int S = 6, P = 2, X = 2;
     int C = 64;
-    while (C > 1 && total(C) > budget) C >>= 1;
-    if (total(C) > budget) return false;
+    for (; C >= 1; C >>= 1) {
+        const int ft = (C + kFinWarps - 1) / kFinWarps;
+        if (ft * cpl > 8) continue;  // z values a finisher lane holds per chunk
+        const size_t t = scan_layout(Ml, C, K, d_v, in_bytes, S, P, X, n, hdr_words_of(kScanWarps, C)).total;
+        if (t <= static_cast<size_t>(kSmemBudget)) break;
+    }
+    if (C < 1) return false;
     out->ncta = n;
+    out->nw = kScanWarps;
+    out->nfin = kFinWarps;
     out->chunk = C;
+    out->stages = S;
+    out->lslots = P;
+    out->xslots = X;
     out->cpl = cpl;
+    out->hdr_words = hdr_words_of(kScanWarps, C);
     out->tmem_cols = alloc;
     // more than half of the SM's shared memory: exactly one CTA (and one TMEM owner) per SM
-    const size_t t = total(C);
+    const size_t t = scan_layout(Ml, C, K, d_v, in_bytes, S, P, X, n, out->hdr_words).total;
+    if (out->ncta * out->nw > 128) return false;
     out->smem_bytes = t < 116 * 1024 ? 116 * 1024 : t;
     return true;
+}
+
+ScanWorkspace scan_workspace(int B, int T, int H, int K, const ScanPlan& plan)
+{
+    ScanWorkspace w;
+    const size_t nch = (static_cast<size_t>(T) + plan.chunk - 1) / plan.chunk;
+    w.events_bytes = static_cast<size_t>(B) * H * nch * 2 * plan.chunk * K * sizeof(uint4);
+    w.hdr_off = (w.events_bytes + 255) & ~static_cast<size_t>(255);
+    w.hdr_bytes = static_cast<size_t>(B) * H * nch * plan.ncta * plan.hdr_words * sizeof(uint32_t);
+    w.total = w.hdr_off + w.hdr_bytes;
+    return w;
 }
 
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream)
 {
     void (*kern)(ScanParams) = nullptr;
-    void (*norm)(ScanParams) = nullptr;
     switch (p.d_v < 32 ? 1 : p.d_v / 32) {
-        case 1: kern = k_scan<1>; norm = k_scan_norm<1>; break;
-        case 2: kern = k_scan<2>; norm = k_scan_norm<2>; break;
-        case 4: kern = k_scan<4>; norm = k_scan_norm<4>; break;
-        case 8: kern = k_scan<8>; norm = k_scan_norm<8>; break;
+        case 1: kern = k_scan<1>; break;
+        case 2: kern = k_scan<2>; break;
+        case 4: kern = k_scan<4>; break;
+        case 8: kern = k_scan<8>; break;
         default: return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(p.B * p.H * p.ncta), kThreads, smem_bytes, stream>>>(p);
-    e = cudaGetLastError();
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
     if (e != cudaSuccess) return e;
-    const size_t n_th = static_cast<size_t>(p.B) * p.T * p.H;
-    norm<<<static_cast<unsigned>((n_th + 7) / 8), 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.H * p.ncta), 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>((p.nw + p.nfin + 1) * 32), 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(p.ncta);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 cudaError_t launch_wait_selftest(uint32_t* status, uint64_t limit_ns, cudaStream_t stream)

@@ -10,9 +10,12 @@
 // How: the scratch is `g_scan_scratch`, a file-scope static device array of
 // RAMNET_NOALLOC_SCRATCH_BYTES bytes, 256-byte aligned.  The first call on a device (that
 // device being current) looks up the array's device address with cudaGetSymbolAddress
-// and caches it; later calls on that device reuse the cached address.  The call then runs
-// the same event-decode and scan kernels as ramnet_scan_forward with that address as the
-// workspace.  Nothing here, or in what it calls, allocates device or host memory.
+// and caches it together with the identity of the current CUDA context; later calls in the
+// same context reuse the cached address, and a call in a new context (after a device reset,
+// or once the primary context was destroyed and created again, which reloads the module)
+// looks it up again.  The call then runs the same route and scan kernels as
+// ramnet_scan_forward with that address as the workspace.  Nothing here, or in what it
+// calls, allocates device or host memory.
 //
 // Contents: nothing in the array has to start at zero.  Each call writes every event the
 // scan reads (event decode) and resets the read accumulator itself before the scan adds
@@ -33,7 +36,40 @@ static __device__ __align__(256) unsigned char g_scan_scratch[RAMNET_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+
+struct CachedScratch {
+    void* addr;
+    unsigned long long ctx_id;  // context the address belongs to (0: unknown)
+};
+CachedScratch g_scratch[kMaxDevices] = {};
+
+// Identity of the calling thread's current CUDA context (driver entry points resolved
+// through the runtime, so the library does not link the driver library itself).  False if
+// there is no current context or the driver does not provide the calls.
+bool current_context_id(unsigned long long* id)
+{
+    using GetCurrent = int (*)(void**);
+    using GetId = int (*)(void*, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static bool resolved = false;
+    if (!resolved) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess && cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) ==
+                                                     cudaSuccess && q2 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrent>(f1);
+            get_id = reinterpret_cast<GetId>(f2);
+        }
+        resolved = true;
+    }
+    if (get_current == nullptr || get_id == nullptr) return false;
+    void* ctx = nullptr;
+    if (get_current(&ctx) != 0 || ctx == nullptr) return false;
+    return get_id(ctx, id) == 0 && *id != 0;
+}
 
 }  // namespace
 
@@ -58,15 +94,21 @@ extern "C" ramnet_status ramnet_scan_forward_noalloc(const ramnet_config* cfg, i
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_scratch_mutex);
-        if (g_scratch_addr[dev] == nullptr) {
+        unsigned long long id = 0;
+        const bool have_id = current_context_id(&id);
+        CachedScratch& cs = g_scratch[dev];
+        if (cs.addr == nullptr || !have_id || cs.ctx_id != id) {
             void* addr = nullptr;
             e = cudaGetSymbolAddress(&addr, g_scan_scratch);
             if (e != cudaSuccess || addr == nullptr)
                 return ramnet::set_last_error(RAMNET_ERR_CUDA, e != cudaSuccess ? cudaGetErrorString(e)
                                                                                  : "static scratch has no address");
-            g_scratch_addr[dev] = addr;
+            // the lookup makes the device's context current if there was none yet
+            unsigned long long id2 = 0;
+            cs.addr = addr;
+            cs.ctx_id = current_context_id(&id2) ? id2 : 0ull;
         }
-        scratch = g_scratch_addr[dev];
+        scratch = cs.addr;
     }
     // 0 means invalid arguments: ramnet_scan_forward reports which one
     const size_t need = ramnet_scan_workspace_bytes(cfg, B, T, H);

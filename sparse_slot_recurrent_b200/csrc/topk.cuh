@@ -139,10 +139,107 @@ __host__ __device__ __forceinline__ void merge_top(uint64_t (&a)[N], const uint6
             if ((i & d) == 0) cx_desc(a[i], a[i + d]);
 }
 
-// One level of the search with the kept list in registers (N = 8 or 16 >= K).  Digit j's
-// candidates f_i + e_j (f_i the extended kept prefix i < nk, descending in i) form a
-// descending list; invalid entries are 0, below every real candidate (a real word is at
-// least 2^48).  The lists are merged one after another into the N best, descending.
+// Both descending lists of N merged into one descending list of 2N: a followed by reversed
+// b is bitonic, and the bitonic merge of size 2N sorts it.
+template <int N>
+__host__ __device__ __forceinline__ void merge_full(const uint64_t (&a)[N], const uint64_t (&b)[N], uint64_t (&out)[2 * N])
+{
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        out[i] = a[i];
+        out[N + i] = b[N - 1 - i];
+    }
+#pragma unroll
+    for (int d = N; d > 0; d >>= 1)
+#pragma unroll
+        for (int i = 0; i < 2 * N; ++i)
+            if ((i & d) == 0) cx_desc(out[i], out[i + d]);
+}
+
+constexpr int pow2_at_least(int x) { return x <= 1 ? 1 : 2 * pow2_at_least((x + 1) / 2); }
+constexpr int int_max(int a, int b) { return a > b ? a : b; }
+
+// Pruned merge of one level.  With the digit codes e sorted best first and the extended
+// kept prefixes f best first, candidate (i, j) = f[i] + e[j] is beaten by every (i', j')
+// with i' <= i, j' <= j, so it can be among the N best only if (i + 1)(j + 1) <= N: digit
+// list j needs only its first N / (j + 1) entries, and lists j >= N none.  The N best form
+// a staircase (n_0 >= n_1 >= ... entries taken from lists 0, 1, ...), so of DE lists the
+// lists j..DE-1 together hold at most N (DE - j) / DE of them.  The lists are merged from
+// the last one backwards, each partial result cut to that bound.  Sizes are powers of two;
+// missing entries are 0, below every real candidate word.  DP is the size of e, DE =
+// min(DP, N) the number of lists that can contribute.
+template <int N, int DP, int DE, int J>
+struct TailMerge {
+    static constexpr int LEN = pow2_at_least(int_max(1, N / (J + 1)));  // entries of list J used
+    static constexpr int SUB = TailMerge<N, DP, DE, J + 1>::SZ;            // size of the merged lists J+1..DE-1
+    static constexpr int X = LEN > SUB ? LEN : SUB;
+    static constexpr int CAP = pow2_at_least(int_max(1, N * (DE - J) / DE));
+    static constexpr bool FULL = 2 * X <= CAP;
+    static constexpr int SZ = FULL ? 2 * X : X;
+
+    __host__ __device__ __forceinline__ static void run(const uint64_t (&f)[N], int nk, const uint64_t (&e)[DP], int d_p,
+                                                        uint64_t (&out)[SZ])
+    {
+        uint64_t sub[X];
+        {
+            uint64_t s[SUB];
+            TailMerge<N, DP, DE, J + 1>::run(f, nk, e, d_p, s);
+#pragma unroll
+            for (int i = 0; i < X; ++i) sub[i] = i < SUB ? s[i < SUB ? i : 0] : 0ull;
+        }
+        uint64_t lst[X];
+#pragma unroll
+        for (int i = 0; i < X; ++i) lst[i] = (i < LEN && i < nk && J < d_p) ? f[i < N ? i : 0] + e[J] : 0ull;
+        if constexpr (FULL) {
+            merge_full<X>(lst, sub, out);
+        } else {
+#pragma unroll
+            for (int i = 0; i < X; ++i) out[i] = lst[i];
+            merge_top<X>(out, sub);
+        }
+    }
+};
+
+template <int N, int DP, int DE>
+struct TailMerge<N, DP, DE, DE - 1> {
+    static constexpr int LEN = pow2_at_least(int_max(1, N / DE));
+    static constexpr int SZ = LEN;
+    __host__ __device__ __forceinline__ static void run(const uint64_t (&f)[N], int nk, const uint64_t (&e)[DP], int d_p,
+                                                        uint64_t (&out)[SZ])
+    {
+#pragma unroll
+        for (int i = 0; i < LEN; ++i) out[i] = (i < nk && DE - 1 < d_p) ? f[i < N ? i : 0] + e[DE - 1] : 0ull;
+    }
+};
+
+// Digit codes of one level sorted best first.  A code is (score << 16) + (d_p - 1 - d) taken
+// as a signed 64-bit number, so that signed order is (score, lower digit) order; digits
+// d >= d_p get INT64_MIN and sort last.  Bitonic sort, DPMAX a power of two.
+template <int DPMAX>
+__host__ __device__ __forceinline__ void sort_codes_desc(uint64_t (&e)[DPMAX])
+{
+#pragma unroll
+    for (int k = 2; k <= DPMAX; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < DPMAX; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const int64_t a = static_cast<int64_t>(e[i]), b = static_cast<int64_t>(e[l]);
+                    const bool swap = ((i & k) == 0) ? (a < b) : (a > b);
+                    if (swap) {
+                        e[i] = static_cast<uint64_t>(b);
+                        e[l] = static_cast<uint64_t>(a);
+                    }
+                }
+            }
+}
+
+// One level of the search with the kept list in registers (N >= K, a power of two).  `e`
+// holds this level's digit codes sorted best first (sort_codes_desc), `kept` the nk best
+// prefixes of the previous level, best first, 0 beyond nk.  On return kept holds the N best
+// candidates of the level, best first (0 where there are fewer).
 template <int N, int DPMAX>
 __host__ __device__ __forceinline__ void topk_level_net(uint64_t (&kept)[N], int nk, const uint64_t (&e)[DPMAX], int d_p)
 {
@@ -150,37 +247,34 @@ __host__ __device__ __forceinline__ void topk_level_net(uint64_t (&kept)[N], int
     uint64_t f[N];
 #pragma unroll
     for (int i = 0; i < N; ++i) f[i] = kept[i] + (kept[i] & 0xFFFFull) * mul;
-    uint64_t acc[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) acc[i] = i < nk ? f[i] + e[0] : 0ull;
-#pragma unroll
-    for (int j = 1; j < DPMAX; ++j) {
-        if (j < d_p) {
-            uint64_t l[N];
-#pragma unroll
-            for (int i = 0; i < N; ++i) l[i] = i < nk ? f[i] + e[j] : 0ull;
-            merge_top<N>(acc, l);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < N; ++i) kept[i] = acc[i];
+    TailMerge<N, DPMAX, (DPMAX < N ? DPMAX : N), 0>::run(f, nk, e, d_p, kept);
 }
 
 // Exact Top-K (K <= N) with the kept list in registers: the same result as topk_search,
-// since the candidate words are distinct and the N best are therefore unique.
+// since the candidate words are distinct and the N best are therefore unique.  Level 0's
+// candidates are the empty prefix extended by each digit, i.e. the sorted digit codes.
 template <int N, int DPMAX>
 __device__ __forceinline__ void topk_search_net(const void* logits, size_t off, int is_bf16, int d_p, int U, int K,
                                                 uint64_t (&out)[N])
 {
     uint64_t kept[N];
-    kept[0] = kKeyBias << 16;  // the empty prefix: score 0, low 0
-#pragma unroll
-    for (int i = 1; i < N; ++i) kept[i] = 0ull;
-    int nk = 1;
-    for (int u = 0; u < U; ++u) {
+    int nk;
+    {
         uint64_t e[DPMAX];
 #pragma unroll
-        for (int d = 0; d < DPMAX; ++d) e[d] = d < d_p ? digit_code(load_in(logits, off + u * d_p + d, is_bf16), d, d_p) : 0ull;
+        for (int d = 0; d < DPMAX; ++d)
+            e[d] = d < d_p ? digit_code(load_in(logits, off + d, is_bf16), d, d_p) : 0x8000000000000000ull;
+        sort_codes_desc<DPMAX>(e);
+        nk = min(K, d_p);
+#pragma unroll
+        for (int i = 0; i < N; ++i) kept[i] = (i < DPMAX && i < nk) ? (kKeyBias << 16) + e[i < DPMAX ? i : 0] : 0ull;
+    }
+    for (int u = 1; u < U; ++u) {
+        uint64_t e[DPMAX];
+#pragma unroll
+        for (int d = 0; d < DPMAX; ++d)
+            e[d] = d < d_p ? digit_code(load_in(logits, off + u * d_p + d, is_bf16), d, d_p) : 0x8000000000000000ull;
+        sort_codes_desc<DPMAX>(e);
         topk_level_net<N, DPMAX>(kept, nk, e, d_p);
         nk = min(K, nk * d_p);
 #pragma unroll

@@ -2,7 +2,8 @@
 
 Argument marshalling only: torch supplies device memory and the current CUDA stream;
 every step of the layer runs in the library's kernels.  The library is loaded from the
-package directory (``libramnet.so``, built by ``build.py``); if it is missing or fails
+package directory (``libramnet.so``, built by ``build.py``; with the environment variable
+RAMNET_DEBUG=1 the range-checking build ``libramnet_debug.so``); if it is missing or fails
 to load, every call raises -- there is no fallback.
 """
 from __future__ import annotations
@@ -14,14 +15,15 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libramnet.so")
+DEBUG = os.environ.get("RAMNET_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libramnet_debug.so" if DEBUG else "libramnet.so")
 
 RAMNET_OK, RAMNET_ERR_INVALID_ARG, RAMNET_ERR_UNSUPPORTED, RAMNET_ERR_CUDA, RAMNET_ERR_TIMEOUT, \
     RAMNET_ERR_DEVICE_CHECK = range(6)
 RAMNET_F32, RAMNET_BF16 = 0, 1
 
 # every symbol include/ramnet.h declares
-EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_forward",
+EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_layout", "ramnet_scan_forward",
             "ramnet_scan_route", "ramnet_scan_recur", "ramnet_scan_forward_noalloc", "ramnet_decode_step",
             "ramnet_selftest_wait_timeout", "ramnet_sync_status", "ramnet_last_error")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # RAMNET_NOALLOC_SCRATCH_BYTES
@@ -31,6 +33,10 @@ class RamnetError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"ramnet status {status}: {msg}")
         self.status = status
+
+
+class _Strides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("t", ctypes.c_int64), ("h", ctypes.c_int64)]
 
 
 class _Cfg(ctypes.Structure):
@@ -72,16 +78,20 @@ def load() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with sparse_slot_recurrent_b200/build.py")
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with sparse_slot_recurrent_b200/build.py"
+                           + (" --debug" if DEBUG else ""))
     lib = ctypes.CDLL(LIB_PATH)
     for name in EXPORTED:
         if not hasattr(lib, name):
             raise RuntimeError(f"{LIB_PATH} does not export {name}")
     C = ctypes.POINTER(_Cfg)
     lib.ramnet_decode_addresses.restype = ctypes.c_int
-    lib.ramnet_decode_addresses.argtypes = [C, _I, _I, _I, _P, ctypes.c_int, _P, _P, _P, _P, _P]
+    lib.ramnet_decode_addresses.argtypes = [C, _I, _I, _I, _P, ctypes.c_int, ctypes.POINTER(_Strides), _P, _P, _P,
+                                            _P, _P]
     lib.ramnet_scan_workspace_bytes.restype = ctypes.c_size_t
     lib.ramnet_scan_workspace_bytes.argtypes = [C, _I, _I, _I]
+    lib.ramnet_scan_layout.restype = ctypes.c_int
+    lib.ramnet_scan_layout.argtypes = [C, ctypes.c_int, _P, _P, _P, _P]
     lib.ramnet_scan_forward.restype = ctypes.c_int
     lib.ramnet_scan_forward.argtypes = [C, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]
@@ -145,22 +155,43 @@ def _dense(*ts):
 
 def decode_addresses(cfg: Config, logits: torch.Tensor, pos0=None, cape_mask=None, idx_out=None, w_out=None,
                      stream=None):
-    """logits [B,T,H,U*d_p] (fp32 or bf16) -> (idx int32 [B,T,H,K], w fp32 [B,T,H,K])."""
+    """logits [B,T,H,U*d_p] (fp32 or bf16; any strides with the last dimension contiguous)
+    -> (idx int32 [B,T,H,K], w fp32 [B,T,H,K])."""
     B, T, H, L = logits.shape
-    _dense(logits, pos0, cape_mask)
+    if logits.stride(-1) != 1:
+        raise ValueError("the last dimension of logits must be contiguous")
+    _dense(pos0, cape_mask)
     if idx_out is None:
         idx_out = torch.empty((B, T, H, cfg.K), dtype=torch.int32, device=logits.device)
     if w_out is None:
         w_out = torch.empty((B, T, H, cfg.K), dtype=torch.float32, device=logits.device)
     c = cfg._c()
-    _check(load().ramnet_decode_addresses(ctypes.byref(c), B, T, H, _ptr(logits), _dt(logits), _ptr(pos0),
-                                          _ptr(cape_mask), _ptr(idx_out), _ptr(w_out), _stream(stream)))
+    st = _Strides(*logits.stride()[:3])
+    _check(load().ramnet_decode_addresses(ctypes.byref(c), B, T, H, _ptr(logits), _dt(logits), ctypes.byref(st),
+                                          _ptr(pos0), _ptr(cape_mask), _ptr(idx_out), _ptr(w_out), _stream(stream)))
     return idx_out, w_out
 
 
 def scan_workspace_bytes(cfg: Config, B: int, T: int, H: int) -> int:
     c = cfg._c()
     return int(load().ramnet_scan_workspace_bytes(ctypes.byref(c), B, T, H))
+
+
+@dataclass(frozen=True)
+class ScanLayout:
+    chunk: int
+    ncta: int
+    scan_warps: int
+    hdr_words: int
+
+
+def scan_layout(cfg: Config, in_dtype=torch.bfloat16) -> ScanLayout:
+    """The prefill's work split for this config and input dtype (see ramnet_scan_layout)."""
+    vals = [ctypes.c_int32() for _ in range(4)]
+    c = cfg._c()
+    dt = RAMNET_BF16 if in_dtype == torch.bfloat16 else RAMNET_F32
+    _check(load().ramnet_scan_layout(ctypes.byref(c), dt, *(ctypes.byref(v) for v in vals)))
+    return ScanLayout(*(v.value for v in vals))
 
 
 def scan_forward(cfg: Config, k_logits, q_logits, v, g, z, norm_w=None, cape_mask=None, pos0=None, S_in=None,

@@ -1,5 +1,5 @@
-// Host-side check of the register Top-K level merge (topk_level_net in topk.cuh) against a
-// plain sort of all candidates.  Built and run by tests/test_topk_net_host.py; prints
+// Host-side check of the register Top-K level merge (sort_codes_desc + topk_level_net in
+// topk.cuh, the pruned merge tree) against a plain sort of all candidates.  Built and run by tests/test_topk_net_host.py; prints
 // "checked <n> mismatches <m>" and exits non-zero on any mismatch.
 #include <algorithm>
 #include <cstdint>
@@ -28,7 +28,8 @@ static long check(std::mt19937_64& rng, long trials, long& n)
         uint64_t kept[N] = {0};
         for (int i = 0; i < nk; ++i) kept[i] = kv[i];
         // digit codes, with repeated scores to exercise the index tie-break
-        uint64_t e[DPMAX] = {0};
+        uint64_t e[DPMAX];
+        for (int d = 0; d < DPMAX; ++d) e[d] = 0x8000000000000000ull;  // digits beyond d_p
         for (int d = 0; d < d_p; ++d) {
             int64_t q = static_cast<int64_t>(rng() % 200001) - 100000;
             if (d > 0 && rng() % 6 == 0) q = static_cast<int64_t>(e[d - 1]) >> 16;
@@ -40,6 +41,7 @@ static long check(std::mt19937_64& rng, long trials, long& n)
                 cand.push_back(kept[i] + (kept[i] & 0xFFFFull) * static_cast<uint64_t>(d_p - 1) + e[d]);
         std::sort(cand.rbegin(), cand.rend());
         const int nout = std::min(K, nk * d_p);
+        ramnet::sort_codes_desc<DPMAX>(e);
         ramnet::topk_level_net<N, DPMAX>(kept, nk, e, d_p);
         for (int i = 0; i < nout; ++i) {
             ++n;
@@ -58,6 +60,9 @@ int main()
     bad += check<16, 4>(rng, 20000, n);
     bad += check<16, 8>(rng, 20000, n);
     bad += check<16, 16>(rng, 20000, n);
+    bad += check<8, 16>(rng, 20000, n);
+    bad += check<32, 4>(rng, 20000, n);
+    bad += check<32, 8>(rng, 10000, n);
     std::printf("checked %ld mismatches %ld\n", n, bad);
     return bad != 0;
 }

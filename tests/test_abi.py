@@ -48,9 +48,10 @@ def _cfg(**kw):
 FAKE = 1 << 40  # 16-byte aligned, never dereferenced: every call below fails host-side
 
 
-def _decode(lib, cfg, B=1, T=4, H=1, logits=FAKE, dt=ramnet.RAMNET_BF16, idx=FAKE, w=FAKE, pos0=None):
+def _decode(lib, cfg, B=1, T=4, H=1, logits=FAKE, dt=ramnet.RAMNET_BF16, idx=FAKE, w=FAKE, pos0=None, strides=None):
     c = cfg._c()
-    return lib.ramnet_decode_addresses(ctypes.byref(c), B, T, H, logits, dt, pos0, None, idx, w, None)
+    st = None if strides is None else ctypes.byref(ramnet._Strides(*strides))
+    return lib.ramnet_decode_addresses(ctypes.byref(c), B, T, H, logits, dt, st, pos0, None, idx, w, None)
 
 
 @pytest.mark.parametrize("kw", [dict(d_p=1), dict(d_p=17), dict(U=0), dict(U=9), dict(d_p=16, U=5),
@@ -65,8 +66,12 @@ def test_bad_pointers_and_sizes_rejected(lib):
     cfg = _cfg()
     assert _decode(lib, cfg, logits=None) == ramnet.RAMNET_ERR_INVALID_ARG
     assert "logits" in ramnet.last_error()
-    assert _decode(lib, cfg, logits=FAKE + 4) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _decode(lib, cfg, logits=FAKE + 1) == ramnet.RAMNET_ERR_INVALID_ARG
     assert "aligned" in ramnet.last_error()
+    assert _decode(lib, cfg, logits=FAKE + 2, dt=ramnet.RAMNET_F32) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert _decode(lib, cfg, strides=(80, -20, 20)) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert "stride" in ramnet.last_error()
+    assert _decode(lib, cfg, idx=FAKE + 4) == ramnet.RAMNET_ERR_INVALID_ARG
     assert _decode(lib, cfg, idx=None) == ramnet.RAMNET_ERR_INVALID_ARG
     assert _decode(lib, cfg, pos0=FAKE + 8) == ramnet.RAMNET_ERR_INVALID_ARG
     assert _decode(lib, cfg, B=0) == ramnet.RAMNET_ERR_INVALID_ARG
@@ -124,15 +129,35 @@ def test_valid_call_without_device_reports_cuda_error(lib):
     assert ramnet.last_error() != ""
 
 
-def test_scan_workspace_is_events_then_accumulator(lib):
-    # decoded events (16 bytes each, 2*K per token-head), then the fp32 read accumulator
-    # at a 256-byte boundary
+def test_scan_workspace_is_events_then_headers(lib):
+    # decoded events (16 bytes each, 2*K per token, grouped in chunks of C tokens), then one
+    # header per (head, chunk, rank) at a 256-byte boundary; the larger of the two input
+    # dtypes' plans
     for (d_p, U, K, d_v), (B, T, H) in [((4, 5, 8, 128), (8, 4096, 8)), ((3, 5, 7, 32), (1, 77, 2)),
-                                         ((16, 2, 64, 256), (2, 33, 3))]:
-        c = _cfg(d_p=d_p, U=U, K=K, d_v=d_v)._c()
-        events = B * H * T * 2 * K * 16
-        o_off = (events + 255) // 256 * 256
-        assert lib.ramnet_scan_workspace_bytes(ctypes.byref(c), B, T, H) == o_off + B * T * H * d_v * 4
+                                         ((16, 2, 64, 256), (2, 33, 3)), ((4, 5, 32, 128), (8, 8192, 8))]:
+        cfg = _cfg(d_p=d_p, U=U, K=K, d_v=d_v)
+        c = cfg._c()
+        want = 0
+        for dt in (torch.bfloat16, torch.float32):
+            lay = ramnet.scan_layout(cfg, dt)
+            assert lay.chunk >= 1 and lay.chunk & (lay.chunk - 1) == 0 and 64 % lay.chunk == 0
+            assert lay.ncta in (1, 2, 4, 8) and lay.scan_warps == 16 and lay.hdr_words % 4 == 0
+            assert lay.hdr_words >= 4 + lay.scan_warps + 1 + (lay.chunk + 3) // 4
+            nch = -(-T // lay.chunk)
+            events = B * H * nch * 2 * lay.chunk * K * 16
+            want = max(want, (events + 255) // 256 * 256 + B * H * nch * lay.ncta * lay.hdr_words * 4)
+        assert lib.ramnet_scan_workspace_bytes(ctypes.byref(c), B, T, H) == want
+
+
+def test_scan_layout_checks(lib):
+    c = _cfg()._c()
+    out = [ctypes.c_int32() for _ in range(4)]
+    assert lib.ramnet_scan_layout(ctypes.byref(c), 9, *(ctypes.byref(v) for v in out)) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert lib.ramnet_scan_layout(ctypes.byref(c), ramnet.RAMNET_BF16, None, *(ctypes.byref(v) for v in out[1:])) == \
+        ramnet.RAMNET_ERR_INVALID_ARG
+    big = _cfg(d_p=16, U=4, K=8, d_v=256)._c()
+    assert lib.ramnet_scan_layout(ctypes.byref(big), ramnet.RAMNET_BF16, *(ctypes.byref(v) for v in out)) == \
+        ramnet.RAMNET_ERR_UNSUPPORTED
 
 
 def test_two_launch_form_checks(lib):

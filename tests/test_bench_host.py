@@ -83,4 +83,4 @@ def test_reference_arm_prints_json_line():
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
-    assert line["config"]["workload"] == "prefill_340m_top8"
+    assert line["config"]["workload"] == "prefill_1p3b_top16"

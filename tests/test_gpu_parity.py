@@ -97,6 +97,25 @@ def test_decode_addresses_matches_oracle(d_p, U, K, dtype, mode):
     del cfg, ocfg
 
 
+def test_decode_addresses_strided_views():
+    """Logits handed over as non-contiguous views (ramnet_strides): a [B,H,T,L] array read as
+    [B,T,H,L], and a slice of wider rows starting at an odd element."""
+    d_p, U, K = 4, 5, 16
+    cfg = ramnet.Config(d_p=d_p, U=U, K=K, d_v=16)
+    ocfg = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=16)
+    B, T, H, L = 2, 45, 3, d_p * U
+    pos0 = torch.tensor([7, 100], dtype=torch.int32)
+    mask = torch.tensor([1, 0, 1], dtype=torch.uint8)
+    base = _logits(B, H, T, L, "ties", torch.bfloat16, seed=77).cuda()  # [B,H,T,L]
+    wide = _logits(B, T, H, L + 9, "normal", torch.bfloat16, seed=78).cuda()
+    for xd in (base.permute(0, 2, 1, 3), wide[..., 3:3 + L]):
+        assert not xd.is_contiguous() and xd.stride(-1) == 1
+        idx, w = ramnet.decode_addresses(cfg, xd, pos0=pos0.cuda(), cape_mask=mask.cuda())
+        oi, ow = oracle.decode_addresses(ocfg, xd.cpu().contiguous(), pos0=pos0, cape_mask=mask)
+        assert np.array_equal(idx.cpu().numpy(), oi)
+        assert _maxabs(w, ow) <= 2e-6
+
+
 @pytest.mark.parametrize("name", ["prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16"])
 def test_decode_addresses_full_size_sampled(name):
     w = WORKLOADS[name]
@@ -206,7 +225,8 @@ def test_scan_raw_product_softmax_weights():
 
 def test_scan_route_then_recur_matches_oracle_and_forward():
     """The two-launch form (route, then recurrence over the workspace) gives the oracle's
-    results and the single-call results (the state exactly)."""
+    results and, bit for bit, the single-call results; a second recurrence over the same
+    workspace gives the same bits again (every sum on the path has a fixed order)."""
     w, inp = _small_inputs(4, 4, 16, 64, 2, 233, 2, torch.bfloat16, "normal", seed=21)
     cfg, ocfg = _cfgs(w)
     g = torch.Generator().manual_seed(22)
@@ -223,10 +243,12 @@ def test_scan_route_then_recur_matches_oracle_and_forward():
     ramnet.sync_status()
     oy, oS, om = _oracle_scan(ocfg, inp, None, S_in, m_in)
     assert _maxabs(y, oy) <= TOL_BF16 and _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
-    # the state is computed in a fixed order and comes out identical; y adds its K read rows
-    # in whatever order they arrive, so it agrees to rounding
     assert torch.equal(S.cpu(), S0.cpu()) and torch.equal(m.cpu(), m0.cpu())
-    assert _maxabs(y, y0) <= TOL_F32
+    assert torch.equal(y.cpu(), y0.cpu())
+    y2, S2, m2 = torch.full_like(y, float("nan")), torch.full_like(S, float("nan")), torch.full_like(m, float("nan"))
+    ramnet.scan_recur(cfg, d["v"], d["z"], y2, S2, m2, ws, S_in=S_in.cuda(), m_in=m_in.cuda())
+    ramnet.sync_status()
+    assert torch.equal(y2, y) and torch.equal(S2, S) and torch.equal(m2, m)
 
 
 def test_scan_unselected_slots_bit_identical():
@@ -250,13 +272,17 @@ def test_scan_unselected_slots_bit_identical():
 
 
 def test_scan_bf16_output_is_rounded_fp32_output():
+    """Every bf16 output element is the round-to-nearest-even of the fp32 output element of
+    the same call (the path is deterministic), and the fp32 output is within tolerance of the
+    oracle, so each bf16 element is within one bf16 rounding of the oracle's value."""
     w, inp = _small_inputs(4, 5, 8, 128, 1, 130, 2, torch.bfloat16, "off", seed=6)
     cfg, ocfg = _cfgs(w)
-    yb, _, _ = _gpu_scan(cfg, inp, out_dtype=torch.bfloat16)
+    yb, Sb, mb = _gpu_scan(cfg, inp, out_dtype=torch.bfloat16)
+    yf, Sf, mf = _gpu_scan(cfg, inp, out_dtype=torch.float32)
+    assert torch.equal(yb, yf.to(torch.bfloat16))
+    assert torch.equal(Sb, Sf) and torch.equal(mb, mf)
     oy, _, _ = _oracle_scan(ocfg, inp)
-    oy = torch.from_numpy(oy)
-    # one bf16 rounding of a value within the bf16-input tolerance
-    assert (yb.double() - oy).abs().max() <= TOL_BF16 + 2.0 ** -8 * oy.abs().max()
+    assert _maxabs(yf, oy) <= TOL_BF16
 
 
 def test_scan_state_carry_matches_single_call():
@@ -301,6 +327,247 @@ def test_scan_full_size_sampled_heads(name):
     written[bi.reshape(-1), hi.reshape(-1), idx.reshape(-1).long()] = True
     written = written.cpu()
     assert (S[~written] == 0).all() and (m[~written] == 0).all()
+
+
+def _parse_route_workspace(cfg, dtype, ws, B, T, H):
+    """Split the workspace written by ramnet_scan_route into per-head event arrays (see
+    ramnet_scan_layout) and check its structure: per chunk the ranks' ranges tile the chunk's
+    events, every event sits in the range of the scan warp that owns its slot, and each
+    owner's events are in (token, stream) order."""
+    lay = ramnet.scan_layout(cfg, dtype)
+    C, ncta, nw, hw, K = lay.chunk, lay.ncta, lay.scan_warps, lay.hdr_words, cfg.K
+    nch = -(-T // C)
+    raw = ws.cpu().numpy()
+    ev_bytes = B * H * nch * 2 * C * K * 16
+    ev = raw[:ev_bytes].view(np.uint32).reshape(B * H, nch, 2 * C * K, 4)
+    off = (ev_bytes + 255) // 256 * 256
+    hdr = raw[off:off + B * H * nch * ncta * hw * 4].view(np.uint32).reshape(B * H, nch, ncta, hw)
+    heads = {}
+    for bh in range(B * H):
+        rows = []
+        nloc = np.zeros((nch * C, ncta), np.int64)
+        for c in range(nch):
+            nt = min(C, T - c * C)
+            pos = 0
+            for r in range(ncta):
+                hd = hdr[bh, c, r]
+                start, n = int(hd[0]), int(hd[1])
+                assert start == pos and int(hd[2]) == nt and int(hd[3]) == 0
+                pos += n
+                woff = hd[4:4 + nw + 1].astype(np.int64)
+                assert woff[0] == 0 and woff[-1] == n and np.all(np.diff(woff) >= 0)
+                nloc[c * C:c * C + nt, r] = hd[4 + nw + 1:].view(np.uint8)[:nt]
+                for wi in range(nw):
+                    e = ev[bh, c, start + woff[wi]:start + woff[wi + 1]]
+                    x = e[:, 0].astype(np.int64)
+                    s, tl, q, st = x & 0xFFFF, (x >> 16) & 0xFF, (x >> 24) & 0x3F, x >> 31
+                    slot = e[:, 3].astype(np.int64)
+                    assert np.all(slot % ncta == r) and np.all(slot // ncta == s) and np.all(s % nw == wi)
+                    assert np.all(tl < nt)
+                    key = tl * 2 + st
+                    assert np.all(np.diff(key) >= 0), "owner list out of (token, stream) order"
+                    wt = e[:, 1].view(np.float32)
+                    al = e[:, 2].view(np.float32)
+                    ints = np.stack([c * C + tl, st, slot, q, np.full_like(tl, r)], 1).astype(np.int64)
+                    rows.append((ints, wt.astype(np.float64), al.astype(np.float64)))
+            assert pos == 2 * nt * K
+        ints = np.concatenate([r[0] for r in rows])
+        heads[bh] = (ints, np.concatenate([r[1] for r in rows]), np.concatenate([r[2] for r in rows]), nloc)
+    return heads, ncta
+
+
+def _check_route_head(ocfg, heads, ncta, bh, k_logits, q_logits, g, pos, cape_on, K):
+    """One head's events against the oracle: write and read slot sets bit for bit, the
+    per-rank read order (q) equal to the oracle's rank order, weights, retentions, and the
+    per-rank read counts."""
+    ints, wt, al, nloc = heads[bh]
+    T = k_logits.shape[0]
+    mask = np.array([1 if cape_on else 0], np.uint8)
+    oi_k, ow_k = oracle.decode_addresses(ocfg, k_logits.reshape(1, T, 1, -1), pos0=np.array([pos], np.int32),
+                                         cape_mask=mask)
+    oi_q, ow_q = oracle.decode_addresses(ocfg, q_logits.reshape(1, T, 1, -1), pos0=np.array([pos], np.int32),
+                                         cape_mask=mask)
+    oi_k, ow_k, oi_q, ow_q = oi_k[0, :, 0], ow_k[0, :, 0], oi_q[0, :, 0], ow_q[0, :, 0]
+    tok, st, slot, q, rk = ints.T
+    # writes: per token the same slots (sorted), with the same weights
+    wsel = st == 0
+    o = np.lexsort((slot[wsel], tok[wsel]))
+    osort = np.argsort(oi_k, axis=1, kind="stable")
+    assert np.array_equal(slot[wsel][o], np.take_along_axis(oi_k, osort, 1).reshape(-1))
+    exp_w = np.take_along_axis(ow_k, osort, 1).reshape(-1)
+    assert np.abs(wt[wsel][o] - exp_w).max() <= 2e-6
+    # retention of GSU step 1 from the same (fp32) weight and the token's gate
+    gw = np.repeat(g.astype(np.float64), K)
+    a_gpu, w_gpu = al[wsel][o], wt[wsel][o]
+    for i in range(0, exp_w.size, max(1, exp_w.size // 3000)):
+        assert abs(a_gpu[i] - oracle.alpha(w_gpu[i], gw[i])) <= 4e-6
+    # reads: per token and rank, in q order, the oracle's reads of that rank in rank (j) order
+    rsel = st == 1
+    o = np.lexsort((q[rsel], rk[rsel], tok[rsel]))
+    ork = oi_q % ncta
+    osort = np.argsort(ork, axis=1, kind="stable")
+    assert np.array_equal(slot[rsel][o], np.take_along_axis(oi_q, osort, 1).reshape(-1))
+    assert np.abs(wt[rsel][o] - np.take_along_axis(ow_q, osort, 1).reshape(-1)).max() <= 2e-6
+    assert np.all(al[rsel] == 0.0)
+    cnt = np.stack([(ork == r).sum(1) for r in range(ncta)], 1)
+    assert np.array_equal(nloc[:T], cnt)
+
+
+ROUTE_CASES = [
+    # d_p, U, K, d_v, B, T, H, dtype, logit mode, cape
+    (4, 5, 8, 128, 1, 200, 2, torch.bfloat16, "normal", "mixed"),
+    (4, 5, 8, 128, 1, 97, 1, torch.bfloat16, "ties", "all"),
+    (4, 5, 16, 128, 1, 150, 2, torch.bfloat16, "ties", "off"),
+    (4, 5, 32, 128, 1, 70, 1, torch.bfloat16, "mixed", "all"),
+    (8, 4, 16, 128, 1, 40, 1, torch.bfloat16, "normal", "all"),
+    (3, 4, 17, 32, 1, 60, 2, torch.float32, "ties", "mixed"),
+    (2, 8, 64, 16, 1, 33, 1, torch.float32, "normal", "off"),
+]
+
+
+@pytest.mark.parametrize("case", ROUTE_CASES)
+def test_route_events_match_oracle(case):
+    """ramnet_scan_route's workspace, decoded: the hot path's Top-K (the register search for
+    K <= 32), weights, CAPE and retentions bit-exact / within 2e-6 of the oracle, and the
+    events bucketed by owning scan warp in causal order."""
+    d_p, U, K, d_v, B, T, H, dtype, mode, cape = case
+    cfg = ramnet.Config(d_p=d_p, U=U, K=K, d_v=d_v)
+    ocfg = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=d_v)
+    kx = _logits(B, T, H, d_p * U, mode, dtype, seed=K * 7 + d_p)
+    qx = _logits(B, T, H, d_p * U, mode, dtype, seed=K * 7 + d_p + 1)
+    gg = torch.sigmoid(torch.randn((B, T, H), generator=torch.Generator().manual_seed(K))).to(dtype)
+    mask = torch.tensor([1 if (cape == "all" or (cape == "mixed" and h % 2 == 0)) else 0 for h in range(H)],
+                        dtype=torch.uint8)
+    pos0 = torch.arange(B, dtype=torch.int32) * 977 + 5
+    ws = torch.empty(ramnet.scan_workspace_bytes(cfg, B, T, H), dtype=torch.uint8, device="cuda")
+    ramnet.scan_route(cfg, kx.cuda(), qx.cuda(), gg.cuda(), ws, cape_mask=mask.cuda(), pos0=pos0.cuda())
+    ramnet.sync_status()
+    heads, ncta = _parse_route_workspace(cfg, dtype, ws, B, T, H)
+    for b in range(B):
+        for h in range(H):
+            _check_route_head(ocfg, heads, ncta, b * H + h, kx[b, :, h].double().numpy(), qx[b, :, h].double().numpy(),
+                              gg[b, :, h].double().numpy(), int(pos0[b]), bool(mask[h]), K)
+
+
+@pytest.mark.parametrize("name", ["prefill_340m_top8", "prefill_1p3b_top16", "prefill_340m_top32"])
+def test_route_events_full_size_sampled_heads(name):
+    """The full workload through ramnet_scan_route in the bench's launch configuration;
+    two heads' events decoded and compared with the oracle over the whole sequence."""
+    w = WORKLOADS[name]
+    cfg, ocfg = _cfgs(w)
+    inp = generate(w, seed=0)
+    d = _cuda(inp)
+    ws = torch.empty(ramnet.scan_workspace_bytes(cfg, w.B, w.T, w.H), dtype=torch.uint8, device="cuda")
+    ramnet.scan_route(cfg, d["k_logits"], d["q_logits"], d["g"], ws, cape_mask=d["cape_mask"], pos0=d["pos0"])
+    ramnet.sync_status()
+    lay = ramnet.scan_layout(cfg, w.in_dtype)
+    # parse only the sampled heads' part of the workspace
+    nch = -(-w.T // lay.chunk)
+    per_head_ev = nch * 2 * lay.chunk * w.K * 16
+    ev_bytes = w.B * w.H * per_head_ev
+    hdr_off = (ev_bytes + 255) // 256 * 256
+    per_head_hdr = nch * lay.ncta * lay.hdr_words * 4
+    for (b, h) in [(0, 1), (w.B - 1, w.H - 1)]:
+        bh = b * w.H + h
+        sub = torch.cat([ws[bh * per_head_ev:(bh + 1) * per_head_ev],
+                         torch.zeros((-per_head_ev) % 256, dtype=torch.uint8, device="cuda"),
+                         ws[hdr_off + bh * per_head_hdr:hdr_off + (bh + 1) * per_head_hdr]])
+        heads, ncta = _parse_route_workspace(cfg, w.in_dtype, sub, 1, w.T, 1)
+        _check_route_head(ocfg, heads, ncta, 0, inp["k_logits"][b, :, h].double().numpy(),
+                          inp["q_logits"][b, :, h].double().numpy(), inp["g"][b, :, h].double().numpy(),
+                          int(inp["pos0"][b]), bool(inp["cape_mask"][h]), w.K)
+
+
+def test_decode_addresses_extreme_logits():
+    """NaN, +-inf and |x| > 4095 logits: indices bit-exact with the oracle (NaN ranks lowest,
+    values clamp at +-4095); weights compared where every logit of the token is within the
+    clamp range (outside it the clamp enters the GPU weights by definition)."""
+    for (d_p, U, K, dtype) in [(4, 5, 8, torch.float32), (4, 5, 16, torch.bfloat16), (8, 4, 16, torch.float32),
+                               (4, 5, 32, torch.float32)]:
+        B, T, H, L = 1, 300, 2, d_p * U
+        g = torch.Generator().manual_seed(K + d_p)
+        x = torch.randn((B, T, H, L), generator=g) * 2
+        pick = torch.rand((B, T, H, L), generator=g)
+        x = torch.where(pick < 0.05, torch.tensor(float("nan")), x)
+        x = torch.where((pick >= 0.05) & (pick < 0.08), torch.tensor(float("inf")), x)
+        x = torch.where((pick >= 0.08) & (pick < 0.11), torch.tensor(float("-inf")), x)
+        x = torch.where((pick >= 0.11) & (pick < 0.14), torch.tensor(1e6), x)
+        x = torch.where((pick >= 0.14) & (pick < 0.17), torch.tensor(-5000.0), x)
+        x = x.to(dtype)
+        cfg = ramnet.Config(d_p=d_p, U=U, K=K, d_v=16)
+        ocfg = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=16)
+        idx, w = ramnet.decode_addresses(cfg, x.cuda())
+        oi, ow = oracle.decode_addresses(ocfg, x)
+        assert np.array_equal(idx.cpu().numpy(), oi)
+        tame = (x.double().abs() <= 4095).all(-1).numpy()
+        assert tame.sum() > 10
+        assert np.abs(w.cpu().numpy()[tame] - ow[tame]).max() <= 2e-6
+
+
+def test_scan_write_gate_edges():
+    """Write gates exactly 0 (alpha = 1: running mean), exactly 1 (alpha = 0: overwrite) and
+    a mixture, through the whole scan, against the oracle's edge rules."""
+    for mode in ("zero", "one", "mixed"):
+        w, inp = _small_inputs(4, 5, 8, 64, 1, 160, 2, torch.float32, "all", seed=41)
+        gm = inp["g"]
+        if mode == "zero":
+            inp["g"] = torch.zeros_like(gm)
+        elif mode == "one":
+            inp["g"] = torch.ones_like(gm)
+        else:
+            r = torch.rand(gm.shape, generator=torch.Generator().manual_seed(42))
+            inp["g"] = torch.where(r < 0.3, torch.zeros_like(gm), torch.where(r < 0.6, torch.ones_like(gm), gm))
+        cfg, ocfg = _cfgs(w)
+        g2 = torch.Generator().manual_seed(43)
+        S_in = torch.randn((1, 2, w.M, 64), generator=g2)
+        m_in = torch.rand((1, 2, w.M), generator=g2)
+        y, S, m = _gpu_scan(cfg, inp, None, S_in, m_in)
+        oy, oS, om = _oracle_scan(ocfg, inp, None, S_in, m_in)
+        assert _maxabs(y, oy) <= TOL_F32, mode
+        assert _maxabs(S, oS) <= TOL_F32, mode
+        assert _maxabs(m, om) <= TOL_F32, mode
+
+
+def test_scan_state_out_aliases_state_in():
+    """S_out and m_out may be the same buffers as S_in and m_in."""
+    w, inp = _small_inputs(4, 5, 16, 128, 2, 120, 2, torch.bfloat16, "mixed", seed=51)
+    cfg, ocfg = _cfgs(w)
+    g2 = torch.Generator().manual_seed(52)
+    S_in = torch.randn((2, 2, w.M, 128), generator=g2)
+    m_in = torch.rand((2, 2, w.M), generator=g2) * 2
+    d = _cuda(inp)
+    S = S_in.cuda()
+    m = m_in.cuda()
+    y, _, _ = ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"], cape_mask=d["cape_mask"],
+                                  pos0=d["pos0"], S_in=S, m_in=m, S_out=S, m_out=m)
+    ramnet.sync_status()
+    oy, oS, om = _oracle_scan(ocfg, inp, None, S_in, m_in)
+    assert _maxabs(y, oy) <= TOL_BF16 and _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
+
+
+def test_scan_every_slot_selected():
+    """K = M (every slot is written and read by every token) and K = 1."""
+    for (d_p, U, K) in [(2, 2, 4), (4, 1, 4), (4, 3, 1)]:
+        w, inp = _small_inputs(d_p, U, K, 32, 1, 90, 2, torch.float32, "all", seed=K + d_p)
+        cfg, ocfg = _cfgs(w)
+        y, S, m = _gpu_scan(cfg, inp)
+        oy, oS, om = _oracle_scan(ocfg, inp)
+        assert _maxabs(y, oy) <= TOL_F32 and _maxabs(S, oS) <= TOL_F32 and _maxabs(m, om) <= TOL_F32
+
+
+def test_scan_full_size_is_deterministic():
+    """Two calls on the full 340M Top-8 workload give identical bits (y, S, m)."""
+    w = WORKLOADS["prefill_340m_top8"]
+    cfg, _ = _cfgs(w)
+    inp = generate(w, seed=0)
+    d = _cuda(inp)
+    outs = []
+    for _ in range(2):
+        outs.append(ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"],
+                                        cape_mask=d["cape_mask"], pos0=d["pos0"], out_dtype=torch.bfloat16))
+        ramnet.sync_status()
+    for a, b2 in zip(outs[0], outs[1]):
+        assert torch.equal(a, b2)
 
 
 # ------------------------------------------------------------------ decode step

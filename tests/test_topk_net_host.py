@@ -3,7 +3,7 @@ sort of all candidates of a level (RAM-Net project page, exactness paragraph aft
 views: the level's K best are among the extensions of the previous level's K best).
 
 Random kept lists and digit codes, including repeated digit scores (the index tie-break),
-for N in {8, 16} and up to 16 digit values.  Needs nvcc, no GPU.
+for N in {8, 16, 32} and up to 16 digit values.  Needs nvcc, no GPU.
 """
 import os
 import shutil
