@@ -436,6 +436,11 @@ def time_prefill(args, world, rank, local, w, with_e2e: bool):
 def run_gpu(args, world, rank, local):
     from sparse_slot_recurrent_b200 import ramnet
     ramnet.load()
+    if args.no_prefill:  # decode only (profiler captures of the decode step)
+        decode = run_decode(args, world, local)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "decode": decode}), flush=True)
+        return
     head = WORKLOADS[args.workload]
     others = [] if args.only_headline else [n for n in PREFILL_ALL if n != head.name]
     main = time_prefill(args, world, rank, local, head, with_e2e=not args.no_e2e)
@@ -460,6 +465,8 @@ def run_decode(args, world, local):
     """1024 consecutive decode steps of the batched workload, one CUDA graph."""
     from sparse_slot_recurrent_b200 import ramnet
     w = WORKLOADS[DECODE]
+    if args.decode_batch:
+        w = w.with_(B=args.decode_batch)
     cfg = ramnet.Config(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
     dev = torch.device("cuda", local)
     inp = generate(w, seed=0)
@@ -524,6 +531,9 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[k for k, v in WORKLOADS.items() if not v.decode],
                     help="headline prefill workload (default: the 1.3B-like Top-16 long-context layer)")
     ap.add_argument("--only-headline", action="store_true", help="time only the headline prefill workload")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="sequences of the decode workload (default 256; smaller for profiler captures)")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill workloads (decode only)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -1,23 +1,27 @@
-// decode_step.cu -- K3: one autoregressive token per (b,h) against an HBM-resident state.
+// decode_step.cu -- one autoregressive token per (b,h) against an HBM-resident state.
 //
 // RAM-Net project page, GPU-execution paragraph on decoding: the step touches only the
-// slots its token selects and never scans the whole state.  Per (b,h): decode the key and
-// query addresses (Product Softmax Top-K + CAPE), apply the Gated Sparse Update to the K
-// write rows of S and their masses, read the K read rows (after the write), RMSNorm,
+// slots its token selects and never scans the whole state.  Per (b,h) unit: decode the key
+// and query addresses (Product Softmax Top-K + CAPE), apply the Gated Sparse Update to the
+// K write rows of S and their masses, read the K read rows (after the write), RMSNorm,
 // gate, store y.
 //
-// One CTA of 128 threads handles kUnits (b,h) units:
-//   1. warp 0 decodes the kUnits keys (lanes 0..15) and queries (lanes 16..31) at once,
-//      one address per lane, so the integer Top-K search runs on every lane;
-//   2. all threads apply GSU steps 1-3 (retention, mass, rate) to the K write slots of
-//      every unit;
-//   3. warp w takes units w, w+4, ...: lane l owns channels [l*CPL, l*CPL + CPL) of a row,
-//      so a slot row is one coalesced warp access; the K write rows of a unit are loaded
-//      together (16 in flight per lane, 8 at d_v = 256), updated and stored, then its K read rows
-//      are loaded together and summed; RMSNorm by a warp reduction, gate, store y.
-// Write rows of one unit are distinct slots (Top-K without repeats, CAPE a bijection).  A
-// read row loaded by the same lane after its own store of that row sees the stored value
-// (same address, program order), so the read loads follow the write stores directly.
+// One CTA per SM, each over a contiguous range of units, in groups of kGroup units:
+//   decoder warps  lane l decodes stream l / kGroup (key, query) of unit l % kGroup of a
+//                  group: slots, weights and (writes) the retention alpha into a shared-
+//                  memory ring of group slots; the two decoder warps take alternate groups,
+//                  so all decodes of a CTA start at once;
+//   row warps      row warp r takes unit r of every group: it loads the unit's K write
+//                  rows and their K masses together (one DRAM round trip, K rows in flight
+//                  per warp, lane l owning channels [l*CPL, l*CPL + CPL)), runs GSU steps
+//                  1-4 and stores them, then loads the K read rows (a read row equal to a
+//                  write row is the value this lane just stored: same address, program
+//                  order), sums them by weight, RMSNorm, norm weight, gate, y.
+// kRowWarps rows per lane in flight per warp and kRowWarps warps per SM keep about
+// 128 KB of loads outstanding per SM, which is what HBM needs to run at its rate.
+// Write rows of one unit are distinct slots (Top-K without repeats, CAPE a bijection).
+// Group slots are handed over with mbarriers (bounded waits, timeout recorded in the
+// status word).
 #include "common.cuh"
 #include "kernels.h"
 #include "topk.cuh"
@@ -26,132 +30,211 @@ namespace ramnet {
 
 namespace {
 
-constexpr int kStepThreads = 128;
-constexpr int kUnits = 16;     // (b,h) units per CTA
+constexpr int kGroup = 16;       // units per group = lanes per stream of a decoder warp
+constexpr int kRowWarps = kGroup;
+constexpr int kDecWarps = 2;
+constexpr int kSlots = 4;        // group slots in the ring
+constexpr int kStepThreads = (kRowWarps + kDecWarps) * 32;
+
+__device__ __forceinline__ uint64_t now_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait (about 2 s); on expiry records kDevTimeout and raises the CTA's abort flag.
+__device__ __noinline__ void step_wait(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag)
+{
+    if (*abort_flag) return;
+    const uint64_t t_end = now_ns() + 2000000000ull;
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        if (mbar_try(bar, parity)) return;
+        if (now_ns() > t_end || *abort_flag) break;
+    }
+    *abort_flag = 1;
+    set_status(status, kDevTimeout);
+}
+
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// One group slot: per unit the K write slots, weights and retentions, the K read slots and
+// weights.
+template <int KMAX>
+struct GroupSlot {
+    int32_t wi[kGroup][KMAX];
+    float ww[kGroup][KMAX];
+    float wa[kGroup][KMAX];
+    int32_t ri[kGroup][KMAX];
+    float rw[kGroup][KMAX];
+};
 
 template <int KMAX, int DPMAX, int CPL>
-__global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
+__global__ void __launch_bounds__(kStepThreads, 1) k_decode_step(StepParams p)
 {
-    __shared__ uint64_t kept_s[KMAX][32];
-    __shared__ int32_t wi_s[kUnits][KMAX], ri_s[kUnits][KMAX];
-    __shared__ float ww_s[kUnits][KMAX], rw_s[kUnits][KMAX], lam_s[kUnits][KMAX];
     constexpr int kRowBatch = CPL >= 8 ? 8 : 16;  // rows per lane in flight
+    extern __shared__ __align__(16) unsigned char step_smem[];
+    GroupSlot<KMAX>* ring = reinterpret_cast<GroupSlot<KMAX>*>(step_smem);
+    // K > 32 only: the decoders' kept lists, [kDecWarps][KMAX][32]
+    uint64_t* kept_s = reinterpret_cast<uint64_t*>(step_smem + sizeof(GroupSlot<KMAX>) * kSlots);
+    __shared__ uint64_t full[kSlots], empty[kSlots];
+    __shared__ int abort_s;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int L = p.U * p.d_p;
     const int K = p.K, dv = p.d_v, M = p.M;
     const int units = p.B * p.H;
-    const int u0 = blockIdx.x * kUnits;
+    // this CTA's contiguous unit range and its groups
+    const int u_beg = static_cast<int>((static_cast<long long>(units) * blockIdx.x) / gridDim.x);
+    const int u_end = static_cast<int>((static_cast<long long>(units) * (blockIdx.x + 1)) / gridDim.x);
+    const int ngroups = (u_end - u_beg + kGroup - 1) / kGroup;
+    volatile int* abort_flag = &abort_s;
 
-    // ---- 1. address decode: lane l of warp 0 decodes stream l / 16 of unit u0 + l % 16
-    if (warp == 0) {
-        const int ul = lane & (kUnits - 1), stream = lane / kUnits;
-        const int bh = u0 + ul;
-        if (bh < units) {
-            const void* lg = stream == 0 ? p.k_logits : p.q_logits;
-            const size_t off = static_cast<size_t>(bh) * L;
-            uint64_t out[KMAX];
-            if constexpr (KMAX <= 32)
-                topk_search_net<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, out);  // kept list in registers
-            else
-                topk_search<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, &kept_s[0][lane], 32, out);
-            float w[KMAX];
-            topk_weights<KMAX>(out, K, p.renorm, lg, off, p.in_bf16, p.d_p, p.U, w);
-            const int h = bh % p.H, b = bh / p.H;
-            const bool cape = p.cape_mask != nullptr && p.cape_mask[h] != 0;
-            const int64_t pos = p.pos != nullptr ? p.pos[b] : 0;
+    if (tid == 0) {
+        abort_s = 0;
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kRowWarps);
+        }
+        fence_mbar_init_cluster();
+    }
+    __syncthreads();
+
+    if (warp >= kRowWarps) {
+        // ------------------------------------------------------------ decoder warps
+        const int dw = warp - kRowWarps;
+        const int ul = lane & (kGroup - 1), stream = lane / kGroup;
+        const int L = p.U * p.d_p;
+        for (int g = dw; g < ngroups; g += kDecWarps) {
+            const int slot = g % kSlots, use = g / kSlots;
+            if (use >= 1) step_wait(smem_addr(&empty[slot]), (use - 1) & 1, p.status, abort_flag);
+            const int bh = u_beg + g * kGroup + ul;
+            if (bh < u_end && !*abort_flag) {
+                const void* lg = stream == 0 ? p.k_logits : p.q_logits;
+                const size_t off = static_cast<size_t>(bh) * L;
+                uint64_t out[KMAX];
+                if constexpr (KMAX <= 32)
+                    topk_search_net<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, out);  // kept list in registers
+                else
+                    topk_search<KMAX, DPMAX>(lg, off, p.in_bf16, p.d_p, p.U, K, kept_s + (dw * KMAX) * 32 + lane, 32,
+                                             out);
+                float w[KMAX];
+                topk_weights<KMAX>(out, K, p.renorm, lg, off, p.in_bf16, p.d_p, p.U, w);
+                const int h = bh % p.H, b = bh / p.H;
+                const bool cape = p.cape_mask != nullptr && p.cape_mask[h] != 0;
+                const int32_t pm = cape ? cape_shift(0, p.pos != nullptr ? p.pos[b] : 0, M) : 0;
+                const float gg = stream == 0 ? load_in(p.g, bh, p.in_bf16) : 0.0f;
+                GroupSlot<KMAX>& gs = ring[slot];
 #pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (j < K) {
-                    int32_t idx = packed_index(out[j], M);
-                    if (cape) idx = cape_shift(idx, pos, M);
-                    if (!dcheck(idx >= 0 && idx < M, p.status)) idx = 0;
-                    if (stream == 0) {
-                        wi_s[ul][j] = idx;
-                        ww_s[ul][j] = w[j];
-                    } else {
-                        ri_s[ul][j] = idx;
-                        rw_s[ul][j] = w[j];
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < K) {
+                        int32_t idx = packed_index(out[j], M) + pm;
+                        if (idx >= M) idx -= M;
+                        if (!dcheck(idx >= 0 && idx < M, p.status)) idx = 0;
+                        if (stream == 0) {
+                            gs.wi[ul][j] = idx;
+                            gs.ww[ul][j] = w[j];
+                            gs.wa[ul][j] = gsu_alpha(w[j], gg);
+                        } else {
+                            gs.ri[ul][j] = idx;
+                            gs.rw[ul][j] = w[j];
+                        }
                     }
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(smem_addr(&full[slot]));
         }
-    }
-    __syncthreads();
-
-    // ---- 2. GSU steps 1-3: mass and rate of each (distinct) write slot of each unit
-    for (int i = tid; i < kUnits * K; i += kStepThreads) {
-        const int ul = i / K, j = i - ul * K;
-        const int bh = u0 + ul;
-        if (bh < units) {
-            float* mrow = p.m + static_cast<size_t>(bh) * M;
-            const float g = load_in(p.g, bh, p.in_bf16);
-            const int s = wi_s[ul][j];
-            const float w = ww_s[ul][j];
-            const float mn = gsu_alpha(w, g) * mrow[s] + w;
-            mrow[s] = mn;
-            lam_s[ul][j] = w / (mn + p.eps_gsu);
-        }
-    }
-    __syncthreads();
-
-    // ---- 3. content update, read, RMSNorm and gate; one warp per unit at a time
-    const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;  // lanes holding channels
-    const bool act = lane < LW;
-    const int ch0 = (act ? lane : 0) * CPL;
-    float nw[CPL];
+    } else {
+        // ------------------------------------------------------------ row warps
+        const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;  // lanes holding channels
+        const bool act = lane < LW;
+        const int ch0 = (act ? lane : 0) * CPL;
+        float nw[CPL];
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) nw[c] = p.norm_w != nullptr ? p.norm_w[ch0 + c] : 1.0f;
-    for (int ul = warp; ul < kUnits; ul += kStepThreads / 32) {
-        const int bh = u0 + ul;
-        if (bh >= units) break;
-        float* S = p.S + static_cast<size_t>(bh) * M * dv;
-        float vv[CPL], o[CPL];
+        for (int c = 0; c < CPL; ++c) nw[c] = p.norm_w != nullptr ? p.norm_w[ch0 + c] : 1.0f;
+        for (int g = 0; g < ngroups; ++g) {
+            const int slot = g % kSlots, use = g / kSlots;
+            step_wait(smem_addr(&full[slot]), use & 1, p.status, abort_flag);
+            const int bh = u_beg + g * kGroup + warp;
+            if (bh < u_end && !*abort_flag) {
+                const GroupSlot<KMAX>& gs = ring[slot];
+                float* S = p.S + static_cast<size_t>(bh) * M * dv;
+                float* mrow = p.m + static_cast<size_t>(bh) * M;
+                float vv[CPL], zz[CPL], o[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            vv[c] = load_in(p.v, static_cast<size_t>(bh) * dv + ch0 + c, p.in_bf16);
-            o[c] = 0.0f;
-        }
-        for (int j0 = 0; j0 < K; j0 += kRowBatch) {
-            float s[kRowBatch][CPL];
+                for (int c = 0; c < CPL; ++c) {
+                    vv[c] = act ? load_in(p.v, static_cast<size_t>(bh) * dv + ch0 + c, p.in_bf16) : 0.0f;
+                    zz[c] = act ? load_in(p.z, static_cast<size_t>(bh) * dv + ch0 + c, p.in_bf16) : 0.0f;
+                    o[c] = 0.0f;
+                }
+                for (int j0 = 0; j0 < K; j0 += kRowBatch) {
+                    // write rows and their masses in flight together; lane j owns mass j0 + j
+                    float s[kRowBatch][CPL];
 #pragma unroll
-            for (int k = 0; k < kRowBatch; ++k)
-                if (j0 + k < K && act) load_row_g<CPL>(S + static_cast<size_t>(wi_s[ul][j0 + k]) * dv + ch0, s[k]);
+                    for (int k = 0; k < kRowBatch; ++k)
+                        if (j0 + k < K && act) load_row_g<CPL>(S + static_cast<size_t>(gs.wi[warp][j0 + k]) * dv + ch0, s[k]);
+                    const int jm = j0 + lane;
+                    float lam = 0.0f;
+                    if (lane < kRowBatch && jm < K) {
+                        const int sl = gs.wi[warp][jm];
+                        const float w = gs.ww[warp][jm];
+                        const float mn = gs.wa[warp][jm] * mrow[sl] + w;  // GSU steps 1-2
+                        mrow[sl] = mn;
+                        lam = w / (mn + p.eps_gsu);  // step 3
+                    }
 #pragma unroll
-            for (int k = 0; k < kRowBatch; ++k) {
-                if (j0 + k < K && act) {
-                    const float lam = lam_s[ul][j0 + k];
+                    for (int k = 0; k < kRowBatch; ++k) {
+                        const float lk = __shfl_sync(0xffffffffu, lam, k);
+                        if (j0 + k < K && act) {
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) s[k][c] = fmaf(lam, vv[c] - s[k][c], s[k][c]);
-                    store_row_g<CPL>(S + static_cast<size_t>(wi_s[ul][j0 + k]) * dv + ch0, s[k]);
+                            for (int c = 0; c < CPL; ++c) s[k][c] = fmaf(lk, vv[c] - s[k][c], s[k][c]);  // step 4
+                            store_row_g<CPL>(S + static_cast<size_t>(gs.wi[warp][j0 + k]) * dv + ch0, s[k]);
+                        }
+                    }
+                }
+                for (int j0 = 0; j0 < K; j0 += kRowBatch) {
+                    float s[kRowBatch][CPL];
+#pragma unroll
+                    for (int k = 0; k < kRowBatch; ++k)
+                        if (j0 + k < K && act) load_row_g<CPL>(S + static_cast<size_t>(gs.ri[warp][j0 + k]) * dv + ch0, s[k]);
+#pragma unroll
+                    for (int k = 0; k < kRowBatch; ++k) {
+                        if (j0 + k < K && act) {
+                            const float r = gs.rw[warp][j0 + k];
+#pragma unroll
+                            for (int c = 0; c < CPL; ++c) o[c] = fmaf(r, s[k][c], o[c]);
+                        }
+                    }
+                }
+                float ss = 0.0f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) ss = fmaf(o[c], o[c], ss);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float inv = 1.0f / sqrtf(ss / dv + p.eps_norm);
+                if (act) {
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c)
+                        store_out(p.y, static_cast<size_t>(bh) * dv + ch0 + c, o[c] * inv * nw[c] * zz[c], p.out_bf16);
                 }
             }
-        }
-        for (int j0 = 0; j0 < K; j0 += kRowBatch) {
-            float s[kRowBatch][CPL];
-#pragma unroll
-            for (int k = 0; k < kRowBatch; ++k)
-                if (j0 + k < K && act) load_row_g<CPL>(S + static_cast<size_t>(ri_s[ul][j0 + k]) * dv + ch0, s[k]);
-#pragma unroll
-            for (int k = 0; k < kRowBatch; ++k) {
-                if (j0 + k < K && act) {
-                    const float r = rw_s[ul][j0 + k];
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) o[c] = fmaf(r, s[k][c], o[c]);
-                }
-            }
-        }
-        float ss = 0.0f;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) ss = fmaf(o[c], o[c], ss);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = 1.0f / sqrtf(ss / dv + p.eps_norm);
-        if (act) {
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                const size_t e = static_cast<size_t>(bh) * dv + ch0 + c;
-                store_out(p.y, e, o[c] * inv * nw[c] * load_in(p.z, e, p.in_bf16), p.out_bf16);
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(smem_addr(&empty[slot]));
         }
     }
 }
@@ -159,14 +242,26 @@ __global__ void __launch_bounds__(kStepThreads) k_decode_step(StepParams p)
 template <int KMAX, int DPMAX>
 cudaError_t launch_step(const StepParams& p, cudaStream_t s)
 {
-    const unsigned grid = static_cast<unsigned>((p.B * p.H + kUnits - 1) / kUnits);
+    int dev = 0, nsm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int units = p.B * p.H;
+    // one CTA per SM, never fewer than one unit per CTA
+    const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
+    const size_t smem = sizeof(GroupSlot<KMAX>) * kSlots + (KMAX > 32 ? sizeof(uint64_t) * kDecWarps * KMAX * 32 : 0);
+    void (*kern)(StepParams) = nullptr;
     switch (p.d_v < 32 ? 1 : p.d_v / 32) {
-        case 1: k_decode_step<KMAX, DPMAX, 1><<<grid, kStepThreads, 0, s>>>(p); break;
-        case 2: k_decode_step<KMAX, DPMAX, 2><<<grid, kStepThreads, 0, s>>>(p); break;
-        case 4: k_decode_step<KMAX, DPMAX, 4><<<grid, kStepThreads, 0, s>>>(p); break;
-        case 8: k_decode_step<KMAX, DPMAX, 8><<<grid, kStepThreads, 0, s>>>(p); break;
+        case 1: kern = k_decode_step<KMAX, DPMAX, 1>; break;
+        case 2: kern = k_decode_step<KMAX, DPMAX, 2>; break;
+        case 4: kern = k_decode_step<KMAX, DPMAX, 4>; break;
+        case 8: kern = k_decode_step<KMAX, DPMAX, 8>; break;
         default: return cudaErrorInvalidValue;
     }
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kStepThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -33,7 +33,8 @@
 // Every wait is bounded (about 2 s); a wait that gives up records RAMNET_ERR_TIMEOUT in the
 // status word and raises the CTA's abort flag, after which its waits return at once, scan
 // warps skip their events and the loader stops copying, so the kernel ends within seconds.
-// Event fields are checked against their ranges before use (RAMNET_ERR_DEVICE_CHECK).
+// Event fields are clamped into their ranges before use; the RAMNET_DEBUG build also records
+// out-of-range fields (RAMNET_ERR_DEVICE_CHECK).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -387,27 +388,27 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                     float Sv[kBatch][CPL];
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
-                        xk[k] = 0xFFFFFFFFu;
                         if (k < nb) {
                             const uint4 r = evs[e + k];
-                            const int s = static_cast<int>(r.x & 0xFFFFu);
-                            const int tl = static_cast<int>((r.x >> 16) & 0xFFu);
+                            // fields are clamped into range, so even a corrupt workspace cannot
+                            // address outside tensor memory, the stage or the ring; the debug
+                            // build also records the corruption
+                            const int s = min(static_cast<int>(r.x & 0xFFFFu), Ml - 1);
                             const bool rd = (r.x >> 31) != 0u;
-                            const int q = static_cast<int>((r.x >> 24) & 0x3Fu);
-                            if (s < Ml && (s & (NW - 1)) == warp && tl < nt && (!rd || q < K)) {
-                                xk[k] = r.x;
-                                tmem_ld<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), Sv[k]);
-                                const float w = __uint_as_float(r.y);
-                                if (!rd) {
-                                    // GSU steps 1-3: m = alpha*m + w, lambda = w / (m + eps)
-                                    const float mn = fmaf(__uint_as_float(r.z), m_s[s], w);
-                                    m_s[s] = mn;  // every lane stores the same value
-                                    ck[k] = __fdividef(w, mn + p.eps_gsu);
-                                } else {
-                                    ck[k] = w;
-                                }
+                            dcheck(static_cast<int>(r.x & 0xFFFFu) < Ml && (s & (NW - 1)) == warp &&
+                                       static_cast<int>((r.x >> 16) & 0xFFu) < nt &&
+                                       (!rd || static_cast<int>((r.x >> 24) & 0x3Fu) < K),
+                                   p.status);
+                            xk[k] = r.x;
+                            tmem_ld<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), Sv[k]);
+                            const float w = __uint_as_float(r.y);
+                            if (!rd) {
+                                // GSU steps 1-3: m = alpha*m + w, lambda = w / (m + eps)
+                                const float mn = fmaf(__uint_as_float(r.z), m_s[s], w);
+                                m_s[s] = mn;  // every lane stores the same value
+                                ck[k] = __fdividef(w, mn + p.eps_gsu);
                             } else {
-                                set_status(p.status, kDevCheck);
+                                ck[k] = w;
                             }
                         }
                     }
@@ -415,9 +416,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                     bool wrote = false;
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
-                        if (k < nb && xk[k] != 0xFFFFFFFFu) {
-                            const int s = static_cast<int>(xk[k] & 0xFFFFu);
-                            const int tl = static_cast<int>((xk[k] >> 16) & 0xFFu);
+                        if (k < nb) {
+                            const int s = min(static_cast<int>(xk[k] & 0xFFFFu), Ml - 1);
+                            const int tl = min(static_cast<int>((xk[k] >> 16) & 0xFFu), nt - 1);
                             if ((xk[k] >> 31) == 0u) {
                                 // GSU step 4 on the row
                                 float vv[CPL];
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                                 wrote = true;
                             } else {
                                 // read: r * S into the partial ring at (token, q)
-                                const int q = static_cast<int>((xk[k] >> 24) & 0x3Fu);
+                                const int q = min(static_cast<int>((xk[k] >> 24) & 0x3Fu), K - 1);
 #pragma unroll
                                 for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] *= ck[k];
                                 if (lane < LW) sts_row<CPL>(lr + static_cast<size_t>(tl * K + q) * dv, Sv[k]);

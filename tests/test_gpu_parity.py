@@ -487,7 +487,8 @@ def test_decode_addresses_extreme_logits():
         B, T, H, L = 1, 300, 2, d_p * U
         g = torch.Generator().manual_seed(K + d_p)
         x = torch.randn((B, T, H, L), generator=g) * 2
-        pick = torch.rand((B, T, H, L), generator=g)
+        # about half of the tokens get extreme values in some of their logits
+        pick = torch.rand((B, T, H, L), generator=g) + (torch.rand((B, T, H, 1), generator=g) < 0.5).float()
         x = torch.where(pick < 0.05, torch.tensor(float("nan")), x)
         x = torch.where((pick >= 0.05) & (pick < 0.08), torch.tensor(float("inf")), x)
         x = torch.where((pick >= 0.08) & (pick < 0.11), torch.tensor(float("-inf")), x)
@@ -500,7 +501,7 @@ def test_decode_addresses_extreme_logits():
         oi, ow = oracle.decode_addresses(ocfg, x)
         assert np.array_equal(idx.cpu().numpy(), oi)
         tame = (x.double().abs() <= 4095).all(-1).numpy()
-        assert tame.sum() > 10
+        assert tame.sum() > 100 and (~tame).sum() > 100
         assert np.abs(w.cpu().numpy()[tame] - ow[tame]).max() <= 2e-6
 
 
