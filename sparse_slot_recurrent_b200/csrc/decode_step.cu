@@ -57,13 +57,19 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
 }
 
 // Bounded wait (about 2 s); on expiry records kDevTimeout and raises the CTA's abort flag.
-__device__ __noinline__ void step_wait(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag)
+// Between polls the thread sleeps (32 ns doubling to 512 ns), so the row warps waiting for a
+// group leave the issue slots to the decoder warps.
+__device__ __forceinline__ void step_wait(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag)
 {
+    if (mbar_try(bar, parity)) return;
     if (*abort_flag) return;
     const uint64_t t_end = now_ns() + 2000000000ull;
+    uint32_t nap = 32;
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
         if (mbar_try(bar, parity)) return;
         if (now_ns() > t_end || *abort_flag) break;
+        __nanosleep(nap);
+        nap = nap < 512 ? 2 * nap : 512;
     }
     *abort_flag = 1;
     set_status(status, kDevTimeout);

@@ -9,11 +9,12 @@
 // head's cluster, see kernels.h), and within one owner the events stay in (token, stream)
 // order, which is each slot's causal order: a token's writes before its reads.
 //
-// One CTA of 128 threads covers 64 tokens of one head: thread 2*i decodes token i's key
+// One CTA of 128 threads covers 64 tokens of one head: thread i < 64 decodes token i's key
 // (its K events are writes; it also computes the retention alpha of GSU step 1), thread
-// 2*i+1 its query (reads).  The events of each chunk are then placed by a stable counting
-// sort on the owner: per (thread, owner) counts in shared memory, an exclusive prefix over
-// the chunk's threads per owner, and an exclusive prefix over owners per chunk.
+// 64 + i its query (reads), so no warp runs both paths.  The events of each chunk are then
+// placed by a stable counting sort on the owner, rows ordered by (token, stream): per
+// (row, owner) counts in shared memory, an exclusive prefix over the chunk's rows per owner,
+// and an exclusive prefix over owners per chunk.
 #include "common.cuh"
 #include "kernels.h"
 #include "topk.cuh"
@@ -47,7 +48,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     const int nblk_t = (p.T + kRouteTokens - 1) / kRouteTokens;
     const int bh = blockIdx.x / nblk_t, tb = blockIdx.x - (blockIdx.x / nblk_t) * nblk_t;
     const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
-    const int tl_blk = tid >> 1, stream = tid & 1;
+    const int tl_blk = tid & (kRouteTokens - 1), stream = tid / kRouteTokens;
+    const int row_id = tl_blk * 2 + stream;  // (token, stream) order of the counting sort
     const int t = tb * kRouteTokens + tl_blk;
     const bool valid = t < p.T;
     const int ch = tl_blk / C, tl = tl_blk & (C - 1);
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
             if (j < K && dcheck(slot[j] >= 0 && slot[j] < p.M, p.status)) {
                 const int rk = slot[j] & (p.ncta - 1);
                 const int o = (rk << lg_nw) + ((slot[j] >> lg_ncta) & (p.nw - 1));
-                const uint32_t r = atomicAdd(&tc[tid * O + o], 1u);
+                const uint32_t r = atomicAdd(&tc[row_id * O + o], 1u);
                 meta[j] = static_cast<uint32_t>(o) | (r << 16);
                 qv[j] = static_cast<uint32_t>((cnt >> (8 * rk)) & 0xFFull);
                 cnt += 1ull << (8 * rk);
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
         for (int j = 0; j < KMAX; ++j) {
             if (j < K && dcheck(slot[j] >= 0 && slot[j] < p.M && static_cast<int>(meta[j] & 0xFFFFu) < O, p.status)) {
                 const uint32_t o = meta[j] & 0xFFFFu;
-                const uint32_t pos = row[o] + tc[tid * O + o] + (meta[j] >> 16);
+                const uint32_t pos = row[o] + tc[row_id * O + o] + (meta[j] >> 16);
                 if (!dcheck(pos < static_cast<uint32_t>(2 * C * K), p.status)) continue;
                 const uint32_t s = static_cast<uint32_t>(slot[j]) >> lg_ncta;
                 const uint32_t x = s | (static_cast<uint32_t>(tl) << 16) | ((stream ? qv[j] : 0u) << 24) |

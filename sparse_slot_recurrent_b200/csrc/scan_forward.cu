@@ -106,35 +106,55 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// One try_wait on phase `parity` (acquire at cluster scope): the thread is suspended in
-// hardware until the phase completes or about kSuspendNs have passed.
+// One try_wait on phase `parity`: the thread may be suspended in hardware until the phase
+// completes or about kSuspendNs have passed.  CLUSTER selects acquire at cluster scope (for
+// barriers that peers of the cluster arrive on after writing into this CTA's shared memory);
+// otherwise the default CTA scope.
 constexpr uint32_t kSuspendNs = 100000;
 
-__device__ __forceinline__ bool try_wait_cta(uint32_t bar, uint32_t parity)
+template <bool CLUSTER>
+__device__ __forceinline__ bool try_wait_phase(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendNs)
-        : "memory");
+    if constexpr (CLUSTER) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(kSuspendNs)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(kSuspendNs)
+            : "memory");
+    }
     return ok != 0;
 }
 
 // Bounded wait for phase `parity` of the mbarrier at shared address `bar`: at most
-// kSpinLimit polls and `limit_ns` (2 s unless given).  On expiry the status word gets
-// kDevTimeout and the CTA's abort flag is raised, after which every later wait of the CTA
-// returns at once, so a kernel that lost a signal still ends within a few seconds.
-__device__ __noinline__ void wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag,
-                                          uint64_t limit_ns = 2000000000ull)
+// kSpinLimit polls and `limit_ns` (2 s unless given).  Between polls the thread sleeps
+// (32 ns doubling to 256 ns), so waiting warps leave the issue slots to working ones.  On
+// expiry the status word gets kDevTimeout and the CTA's abort flag is raised, after which
+// every later wait of the CTA returns at once, so a kernel that lost a signal still ends
+// within a few seconds.
+template <bool CLUSTER>
+__device__ __forceinline__ void wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag,
+                                             uint64_t limit_ns = 2000000000ull)
 {
+    if (try_wait_phase<CLUSTER>(bar, parity)) return;
     if (*abort_flag) return;
     const uint64_t t_end = global_ns() + limit_ns;
+    uint32_t nap = 32;
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
-        if (try_wait_cta(bar, parity)) return;
+        if (try_wait_phase<CLUSTER>(bar, parity)) return;
         if (global_ns() > t_end || *abort_flag) break;
+        __nanosleep(nap);
+        nap = nap < 256 ? 2 * nap : 256;
     }
     *abort_flag = 1;
     set_status(status, kDevTimeout);
@@ -146,9 +166,16 @@ __device__ __noinline__ void drain_copies(uint32_t bar, uint32_t parity)
 {
     const uint64_t t_end = global_ns() + 2000000000ull;
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
-        if (try_wait_cta(bar, parity)) return;
+        if (try_wait_phase<false>(bar, parity)) return;
         if (global_ns() > t_end) return;
+        __nanosleep(256);
     }
+}
+
+// Arrive (release, CTA scope) on a barrier of this CTA.
+__device__ __forceinline__ void arrive_local(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void arrive_expect_tx(uint32_t bar, uint32_t bytes)
@@ -357,9 +384,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
         tmem_wait_st();
         const unsigned lt_mask = (1u << lane) - 1u;
         for (int c = 0; c < nch; ++c) {
-            wait_bounded(bar(BI.sfull + c % S), (c / S) & 1, p.status, abort_flag);
+            wait_bounded<false>(bar(BI.sfull + c % S), (c / S) & 1, p.status, abort_flag);
             const int ls = c % P, kl = c / P;
-            if (kl >= 1) wait_bounded(bar(BI.lfree + ls), (kl - 1) & 1, p.status, abort_flag);
+            if (kl >= 1) wait_bounded<false>(bar(BI.lfree + ls), (kl - 1) & 1, p.status, abort_flag);
             const unsigned char* st = stage(c);
             const uint32_t* hd = reinterpret_cast<const uint32_t*>(st);
             if (!*abort_flag) {
@@ -442,8 +469,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_cluster(map_to_rank(bar(BI.sfree + c % S), static_cast<uint32_t>(rank)));
-                mbar_arrive_cluster(map_to_rank(bar(BI.ldone + ls), static_cast<uint32_t>(rank)));
+                arrive_local(bar(BI.sfree + c % S));
+                arrive_local(bar(BI.ldone + ls));
             }
         }
         // final state of the owned slots
@@ -489,10 +516,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                     }
                 }
             }
-            wait_bounded(bar(BI.ldone + ls), kl & 1, p.status, abort_flag);
+            wait_bounded<false>(bar(BI.ldone + ls), kl & 1, p.status, abort_flag);
             if (ncta > 1) {
-                if (own) wait_bounded(bar(BI.xfull + xs), kx & 1, p.status, abort_flag);
-                else if (kx >= 1) wait_bounded(bar(BI.xfree + f * X + xs), (kx - 1) & 1, p.status, abort_flag);
+                if (own) wait_bounded<true>(bar(BI.xfull + xs), kx & 1, p.status, abort_flag);
+                else if (kx >= 1) wait_bounded<true>(bar(BI.xfree + f * X + xs), (kx - 1) & 1, p.status, abort_flag);
             }
             const float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
             const int xi = rank < f ? rank : rank - 1;  // this CTA's entry in f's exchange slot
@@ -556,7 +583,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             }
             finisher_sync(F * 32);
             if (fw == 0 && lane == 0) {
-                mbar_arrive_cluster(map_to_rank(bar(BI.lfree + ls), static_cast<uint32_t>(rank)));
+                arrive_local(bar(BI.lfree + ls));
                 if (ncta > 1) {
                     if (own) {
                         for (int r2 = 0; r2 < ncta; ++r2)
@@ -588,7 +615,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             const uint32_t first = min(start, static_cast<uint32_t>(cap) - n);
             const int nt = min(C, p.T - c * C);
             if (c >= S) {
-                wait_bounded(bar(BI.sfree + c % S), (c / S - 1) & 1, p.status, abort_flag);
+                wait_bounded<false>(bar(BI.sfree + c % S), (c / S - 1) & 1, p.status, abort_flag);
                 fence_proxy_async();
             }
             if (*abort_flag) continue;
@@ -632,7 +659,7 @@ __global__ void k_wait_selftest(uint32_t* status, uint64_t limit_ns)
         fence_mbar_init_cluster();
     }
     __syncthreads();
-    if (threadIdx.x == 0) wait_bounded(smem_addr(&never), 0, status, &abort_flag, limit_ns);
+    if (threadIdx.x == 0) wait_bounded<false>(smem_addr(&never), 0, status, &abort_flag, limit_ns);
 }
 
 }  // namespace

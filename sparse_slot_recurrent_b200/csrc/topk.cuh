@@ -32,6 +32,17 @@ __device__ __forceinline__ int64_t digit_score(float x)
     return __float2ll_rn(x * 4294967296.0f);  // exact scaling, round half to even
 }
 
+// Bring the token's logit row (U*d_p elements from element `off`) into L1 before the search
+// reads it level by level, so the U levels do not each wait for a DRAM round trip.
+__device__ __forceinline__ void prefetch_logits(const void* logits, size_t off, int is_bf16, int L)
+{
+    const char* b = static_cast<const char*>(logits) + off * (is_bf16 ? 2 : 4);
+    const char* e = b + static_cast<size_t>(L) * (is_bf16 ? 2 : 4) - 1;
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(b));
+    if ((reinterpret_cast<uintptr_t>(b) >> 7) != (reinterpret_cast<uintptr_t>(e) >> 7))
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(e));
+}
+
 __device__ __forceinline__ uint64_t digit_code(float x, int d, int d_p)
 {
     return (static_cast<uint64_t>(digit_score(x)) << 16) + static_cast<uint64_t>(d_p - 1 - d);
@@ -44,6 +55,7 @@ template <int KMAX, int DPMAX>
 __device__ __forceinline__ void topk_search(const void* logits, size_t off, int is_bf16, int d_p, int U, int K,
                                             uint64_t* kept, int stride, uint64_t (&out)[KMAX])
 {
+    prefetch_logits(logits, off, is_bf16, U * d_p);
     int nk = 1;
     kept[0] = kKeyBias << 16;  // the empty prefix: score 0, low 0
     for (int u = 0; u < U; ++u) {
@@ -257,6 +269,7 @@ template <int N, int DPMAX>
 __device__ __forceinline__ void topk_search_net(const void* logits, size_t off, int is_bf16, int d_p, int U, int K,
                                                 uint64_t (&out)[N])
 {
+    prefetch_logits(logits, off, is_bf16, U * d_p);
     uint64_t kept[N];
     int nk;
     {
