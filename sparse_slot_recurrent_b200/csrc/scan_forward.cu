@@ -42,7 +42,6 @@ namespace ramnet {
 
 namespace {
 
-constexpr int kBatch = 8;  // events per TMEM round trip of a scan warp
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
@@ -193,12 +192,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Named barrier of the finisher warps (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void finisher_sync(int nthreads)
-{
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
-
 // CPL consecutive input elements (fp32 or bf16) from shared memory, as fp32.
 template <int CPL>
 __device__ __forceinline__ void load_row(const unsigned char* base, int elem, int is_bf16, float (&v)[CPL])
@@ -316,15 +309,16 @@ constexpr int kFinWarps = 8;
 constexpr int kScanThreads = (kScanWarps + kFinWarps + 1) * 32;
 constexpr int kSmemBudget = 220 * 1024;
 
-template <int CPL>
+template <int CPL, bool BF>
 __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int kZMax = 8;  // z values a finisher lane prefetches per chunk
+    constexpr int kBatch = CPL >= 8 ? 4 : 8;  // events per TMEM round trip of a scan warp
     const int C = p.chunk, dv = p.d_v, ncta = p.ncta, M = p.M, K = p.K, NW = p.nw, F = p.nfin;
     const int S = p.stages, P = p.lslots, X = p.xslots;
     const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;  // lanes holding channels (32 unless d_v = 16)
-    const int es = p.in_bf16 ? 2 : 4;
+    const int es = BF ? 2 : 4;
     const int rank = static_cast<int>(cluster_ctarank());
     const int bh = static_cast<int>(blockIdx.x) / ncta;
     const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
@@ -355,10 +349,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
         }
         for (int i = 0; i < P; ++i) {
             mbar_init(bar_ptr + BI.ldone + i, NW);
-            mbar_init(bar_ptr + BI.lfree + i, 1);
+            mbar_init(bar_ptr + BI.lfree + i, F);
         }
-        for (int i = 0; i < X; ++i) mbar_init(bar_ptr + BI.xfull + i, ncta > 1 ? ncta - 1 : 1);
-        for (int i = 0; i < ncta * X; ++i) mbar_init(bar_ptr + BI.xfree + i, 1);
+        for (int i = 0; i < X; ++i) mbar_init(bar_ptr + BI.xfull + i, ncta > 1 ? (ncta - 1) * F : 1);
+        for (int i = 0; i < ncta * X; ++i) mbar_init(bar_ptr + BI.xfree + i, F);
         fence_mbar_init_cluster();
     }
     if (warp == 0) tmem_alloc(holder, p.tmem_cols);
@@ -402,64 +396,69 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                 float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
                 int e = beg;
                 while (e < end) {
-                    // the longest run of up to kBatch events on distinct slots
+                    // The longest run of up to kBatch events on distinct slots.  Lane k < nb
+                    // decodes event e + k once for the whole warp: its slot's tensor-memory
+                    // address, the row it touches in shared memory and, for a write, GSU steps
+                    // 1-3 (m = alpha*m + w, lambda = w / (m + eps)); the per-event loops below
+                    // only fetch those values with shuffles.
                     const int navail = end - e;
-                    uint32_t sl = 0x10000u + static_cast<uint32_t>(lane);
-                    if (lane < kBatch && lane < navail) sl = evs[e + lane].x & 0xFFFFu;
+                    const bool act = lane < kBatch && lane < navail;
+                    uint4 r = make_uint4(0u, 0u, 0u, 0u);
+                    if (act) r = evs[e + lane];
+                    const uint32_t sl = act ? (r.x & 0xFFFFu) : 0x10000u + static_cast<uint32_t>(lane);
                     const uint32_t peers = __match_any_sync(0xffffffffu, sl);
                     const uint32_t dup = __ballot_sync(0xffffffffu, (peers & lt_mask) != 0u);
                     int nb = min(navail, kBatch);
                     if (dup != 0u) nb = min(nb, __ffs(dup) - 1);
-                    uint32_t xk[kBatch];
-                    float ck[kBatch];
+                    // fields are clamped into range, so even a corrupt workspace cannot address
+                    // outside tensor memory, the stage or the ring; the debug build also records
+                    // the corruption
+                    const int es_ = min(static_cast<int>(r.x & 0xFFFFu), Ml - 1);
+                    const bool rd = (r.x >> 31) != 0u;
+                    const int etl = min(static_cast<int>((r.x >> 16) & 0xFFu), nt - 1);
+                    const int eq = min(static_cast<int>((r.x >> 24) & 0x3Fu), K - 1);
+                    dcheck(lane >= nb || (static_cast<int>(r.x & 0xFFFFu) < Ml && (es_ & (NW - 1)) == warp &&
+                                          static_cast<int>((r.x >> 16) & 0xFFu) < nt &&
+                                          (!rd || static_cast<int>((r.x >> 24) & 0x3Fu) < K)),
+                           p.status);
+                    float eck = __uint_as_float(r.y);
+                    if (lane < nb && !rd) {
+                        const float mn = fmaf(__uint_as_float(r.z), m_s[es_], eck);
+                        m_s[es_] = mn;
+                        eck = __fdividef(eck, mn + p.eps_gsu);
+                    }
+                    const uint32_t eta = tq + static_cast<uint32_t>((es_ >> 2) * CPL);
+                    // row offset in elements (value row of the stage, or read-partial row of the
+                    // ring) with the read flag in bit 31
+                    const uint32_t erow = rd ? (0x80000000u | static_cast<uint32_t>((etl * K + eq) * dv))
+                                             : static_cast<uint32_t>(etl * dv);
+                    uint32_t ta[kBatch];
                     float Sv[kBatch][CPL];
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
-                        if (k < nb) {
-                            const uint4 r = evs[e + k];
-                            // fields are clamped into range, so even a corrupt workspace cannot
-                            // address outside tensor memory, the stage or the ring; the debug
-                            // build also records the corruption
-                            const int s = min(static_cast<int>(r.x & 0xFFFFu), Ml - 1);
-                            const bool rd = (r.x >> 31) != 0u;
-                            dcheck(static_cast<int>(r.x & 0xFFFFu) < Ml && (s & (NW - 1)) == warp &&
-                                       static_cast<int>((r.x >> 16) & 0xFFu) < nt &&
-                                       (!rd || static_cast<int>((r.x >> 24) & 0x3Fu) < K),
-                                   p.status);
-                            xk[k] = r.x;
-                            tmem_ld<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), Sv[k]);
-                            const float w = __uint_as_float(r.y);
-                            if (!rd) {
-                                // GSU steps 1-3: m = alpha*m + w, lambda = w / (m + eps)
-                                const float mn = fmaf(__uint_as_float(r.z), m_s[s], w);
-                                m_s[s] = mn;  // every lane stores the same value
-                                ck[k] = __fdividef(w, mn + p.eps_gsu);
-                            } else {
-                                ck[k] = w;
-                            }
-                        }
+                        ta[k] = __shfl_sync(0xffffffffu, eta, k);
+                        if (k < nb) tmem_ld<CPL>(ta[k], Sv[k]);
                     }
                     tmem_wait_ld();
                     bool wrote = false;
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
+                        const float ck = __shfl_sync(0xffffffffu, eck, k);
+                        const uint32_t row = __shfl_sync(0xffffffffu, erow, k);
                         if (k < nb) {
-                            const int s = min(static_cast<int>(xk[k] & 0xFFFFu), Ml - 1);
-                            const int tl = min(static_cast<int>((xk[k] >> 16) & 0xFFu), nt - 1);
-                            if ((xk[k] >> 31) == 0u) {
+                            if ((row >> 31) == 0u) {
                                 // GSU step 4 on the row
                                 float vv[CPL];
-                                load_row<CPL>(vb, tl * dv + lch, p.in_bf16, vv);
+                                load_row<CPL>(vb, static_cast<int>(row) + lch, BF, vv);
 #pragma unroll
-                                for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] = fmaf(ck[k], vv[cc] - Sv[k][cc], Sv[k][cc]);
-                                tmem_st<CPL>(tq + static_cast<uint32_t>((s >> 2) * CPL), Sv[k]);
+                                for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] = fmaf(ck, vv[cc] - Sv[k][cc], Sv[k][cc]);
+                                tmem_st<CPL>(ta[k], Sv[k]);
                                 wrote = true;
                             } else {
                                 // read: r * S into the partial ring at (token, q)
-                                const int q = min(static_cast<int>((xk[k] >> 24) & 0x3Fu), K - 1);
 #pragma unroll
-                                for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] *= ck[k];
-                                if (lane < LW) sts_row<CPL>(lr + static_cast<size_t>(tl * K + q) * dv, Sv[k]);
+                                for (int cc = 0; cc < CPL; ++cc) Sv[k][cc] *= ck;
+                                if (lane < LW) sts_row<CPL>(lr + (row & 0x7FFFFFFFu), Sv[k]);
                             }
                         }
                     }
@@ -509,7 +508,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                     const int tl = fw + i * F;
                     if (i < ft && tl < nt && lane < LW) {
                         float zz[CPL];
-                        load_row_in<CPL>(p.z, ((static_cast<size_t>(b) * p.T + t0 + tl) * p.H + h) * dv + lch, p.in_bf16,
+                        load_row_in<CPL>(p.z, ((static_cast<size_t>(b) * p.T + t0 + tl) * p.H + h) * dv + lch, BF,
                                          zz);
 #pragma unroll
                         for (int cc = 0; cc < CPL; ++cc) zr[i * CPL + cc] = zz[cc];
@@ -517,11 +516,32 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                 }
             }
             wait_bounded<false>(bar(BI.ldone + ls), kl & 1, p.status, abort_flag);
+            // this CTA's sum of each token's read partials, in q order
+            const float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
+            float o[kZMax];
+#pragma unroll
+            for (int i = 0; i < kZMax / CPL; ++i) {
+                const int tl = fw + i * F;
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) o[i * CPL + cc] = 0.0f;
+                if (i < ft && tl < nt) {
+                    const int n = min(static_cast<int>(nloc_s[ls * C + tl]), K);
+                    for (int q = 0; q < n; ++q) {
+                        float pr[CPL];
+                        lds_row<CPL>(lr + static_cast<size_t>(tl * K + q) * dv, pr);
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) o[i * CPL + cc] += pr[cc];
+                    }
+                }
+            }
+            // the partial-ring slot is free again once every finisher warp has read it; the
+            // scan warps move on without waiting for the exchange between CTAs
+            __syncwarp();
+            if (lane == 0) arrive_local(bar(BI.lfree + ls));
             if (ncta > 1) {
                 if (own) wait_bounded<true>(bar(BI.xfull + xs), kx & 1, p.status, abort_flag);
                 else if (kx >= 1) wait_bounded<true>(bar(BI.xfree + f * X + xs), (kx - 1) & 1, p.status, abort_flag);
             }
-            const float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
             const int xi = rank < f ? rank : rank - 1;  // this CTA's entry in f's exchange slot
             const uint32_t xdst = ncta > 1 && !own
                                       ? map_to_rank(smem_addr(xbuf + static_cast<size_t>(xs) * xslot_floats +
@@ -532,16 +552,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             for (int i = 0; i < kZMax / CPL; ++i) {
                 const int tl = fw + i * F;
                 if (i < ft && tl < nt) {
-                    const int n = min(static_cast<int>(nloc_s[ls * C + tl]), K);
-                    float o[CPL];
-#pragma unroll
-                    for (int cc = 0; cc < CPL; ++cc) o[cc] = 0.0f;
-                    for (int q = 0; q < n; ++q) {
-                        float pr[CPL];
-                        lds_row<CPL>(lr + static_cast<size_t>(tl * K + q) * dv, pr);
-#pragma unroll
-                        for (int cc = 0; cc < CPL; ++cc) o[cc] += pr[cc];
-                    }
                     if (own) {
                         // rank order: peers below this CTA, this CTA, peers above
                         float tot[CPL];
@@ -550,7 +560,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                         for (int r2 = 0; r2 < ncta; ++r2) {
                             if (r2 == rank) {
 #pragma unroll
-                                for (int cc = 0; cc < CPL; ++cc) tot[cc] += o[cc];
+                                for (int cc = 0; cc < CPL; ++cc) tot[cc] += o[i * CPL + cc];
                             } else {
                                 const int xi2 = r2 < rank ? r2 : r2 - 1;
                                 float pr[CPL];
@@ -577,21 +587,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                                          p.out_bf16);
                         }
                     } else if (lane < LW) {
-                        st_cluster_row<CPL>(xdst + static_cast<uint32_t>(tl * dv * 4), o);
+                        float ov[CPL];
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc) ov[cc] = o[i * CPL + cc];
+                        st_cluster_row<CPL>(xdst + static_cast<uint32_t>(tl * dv * 4), ov);
                     }
                 }
             }
-            finisher_sync(F * 32);
-            if (fw == 0 && lane == 0) {
-                arrive_local(bar(BI.lfree + ls));
-                if (ncta > 1) {
-                    if (own) {
-                        for (int r2 = 0; r2 < ncta; ++r2)
-                            if (r2 != rank)
-                                mbar_arrive_cluster(map_to_rank(bar(BI.xfree + rank * X + xs), static_cast<uint32_t>(r2)));
-                    } else {
-                        mbar_arrive_cluster(map_to_rank(bar(BI.xfull + xs), static_cast<uint32_t>(f)));
-                    }
+            // each finisher warp signals its own rows (stores and reads of the warp ordered
+            // before lane 0's release by the warp barrier)
+            __syncwarp();
+            if (ncta > 1 && lane == 0) {
+                if (own) {
+                    for (int r2 = 0; r2 < ncta; ++r2)
+                        if (r2 != rank)
+                            mbar_arrive_cluster(map_to_rank(bar(BI.xfree + rank * X + xs), static_cast<uint32_t>(r2)));
+                } else {
+                    mbar_arrive_cluster(map_to_rank(bar(BI.xfull + xs), static_cast<uint32_t>(f)));
                 }
             }
         }
@@ -721,11 +733,12 @@ ScanWorkspace scan_workspace(int B, int T, int H, int K, const ScanPlan& plan)
 cudaError_t launch_scan(const ScanParams& p, size_t smem_bytes, cudaStream_t stream)
 {
     void (*kern)(ScanParams) = nullptr;
+    const bool bf = p.in_bf16 != 0;
     switch (p.d_v < 32 ? 1 : p.d_v / 32) {
-        case 1: kern = k_scan<1>; break;
-        case 2: kern = k_scan<2>; break;
-        case 4: kern = k_scan<4>; break;
-        case 8: kern = k_scan<8>; break;
+        case 1: kern = bf ? k_scan<1, true> : k_scan<1, false>; break;
+        case 2: kern = bf ? k_scan<2, true> : k_scan<2, false>; break;
+        case 4: kern = bf ? k_scan<4, true> : k_scan<4, false>; break;
+        case 8: kern = bf ? k_scan<8, true> : k_scan<8, false>; break;
         default: return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
