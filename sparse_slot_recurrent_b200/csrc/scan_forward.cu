@@ -306,6 +306,7 @@ __device__ __forceinline__ void store_y(void* y, size_t elem, const float (&v)[C
 
 constexpr int kScanWarps = 16;
 constexpr int kFinWarps = 8;
+constexpr int kFinGroups = 2;
 constexpr int kScanThreads = (kScanWarps + kFinWarps + 1) * 32;
 constexpr int kSmemBudget = 220 * 1024;
 
@@ -313,7 +314,7 @@ template <int CPL, bool BF>
 __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    constexpr int kZMax = 8;  // z values a finisher lane prefetches per chunk
+    constexpr int kZMax = CPL <= 4 ? 16 : 8;  // z values a finisher lane prefetches per chunk
     constexpr int kBatch = CPL >= 8 ? 4 : 8;  // events per TMEM round trip of a scan warp
     const int C = p.chunk, dv = p.d_v, ncta = p.ncta, M = p.M, K = p.K, NW = p.nw, F = p.nfin;
     const int S = p.stages, P = p.lslots, X = p.xslots;
@@ -349,10 +350,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
         }
         for (int i = 0; i < P; ++i) {
             mbar_init(bar_ptr + BI.ldone + i, NW);
-            mbar_init(bar_ptr + BI.lfree + i, F);
+            mbar_init(bar_ptr + BI.lfree + i, F / kFinGroups);
         }
-        for (int i = 0; i < X; ++i) mbar_init(bar_ptr + BI.xfull + i, ncta > 1 ? (ncta - 1) * F : 1);
-        for (int i = 0; i < ncta * X; ++i) mbar_init(bar_ptr + BI.xfree + i, F);
+        for (int i = 0; i < X; ++i) mbar_init(bar_ptr + BI.xfull + i, ncta > 1 ? (ncta - 1) * (F / kFinGroups) : 1);
+        for (int i = 0; i < ncta * X; ++i) mbar_init(bar_ptr + BI.xfree + i, F / kFinGroups);
         fence_mbar_init_cluster();
     }
     if (warp == 0) tmem_alloc(holder, p.tmem_cols);
@@ -486,13 +487,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
         }
     } else if (warp < NW + F) {
         // ============================================================ finisher warps
+        // kFinGroups groups of finisher warps take alternate chunks, so one group's wait for
+        // a peer CTA does not hold up the next chunk; chunk c goes to group c mod kFinGroups,
+        // which divides ncta (or ncta is 1), so every chunk that one CTA finishes, and so
+        // every use of one exchange slot, stays with one group, in chunk order
         const int fw = warp - NW;
+        const int FG = F / kFinGroups, grp = fw / FG, gw = fw - grp * FG;
         const int lch = (lane < LW ? lane : 0) * CPL;
         float nwv[CPL];
 #pragma unroll
         for (int c = 0; c < CPL; ++c) nwv[c] = p.norm_w != nullptr ? p.norm_w[lch + c] : 1.0f;
-        const int ft = (C + F - 1) / F;  // tokens per finisher warp per chunk (ft * CPL <= kZMax)
-        for (int c = 0; c < nch; ++c) {
+        const int ft = (C + FG - 1) / FG;  // tokens per finisher warp per chunk (ft * CPL <= kZMax)
+        for (int c = grp; c < nch; c += kFinGroups) {
             const int ls = c % P, kl = c / P;
             const int f = c % ncta;
             const int xs = (c / ncta) % X, kx = c / (ncta * X);
@@ -505,7 +511,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             if (own) {
 #pragma unroll
                 for (int i = 0; i < kZMax / CPL; ++i) {
-                    const int tl = fw + i * F;
+                    const int tl = gw + i * FG;
                     if (i < ft && tl < nt && lane < LW) {
                         float zz[CPL];
                         load_row_in<CPL>(p.z, ((static_cast<size_t>(b) * p.T + t0 + tl) * p.H + h) * dv + lch, BF,
@@ -521,7 +527,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             float o[kZMax];
 #pragma unroll
             for (int i = 0; i < kZMax / CPL; ++i) {
-                const int tl = fw + i * F;
+                const int tl = gw + i * FG;
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc) o[i * CPL + cc] = 0.0f;
                 if (i < ft && tl < nt) {
@@ -550,7 +556,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                                       : 0u;
 #pragma unroll
             for (int i = 0; i < kZMax / CPL; ++i) {
-                const int tl = fw + i * F;
+                const int tl = gw + i * FG;
                 if (i < ft && tl < nt) {
                     if (own) {
                         // rank order: peers below this CTA, this CTA, peers above
@@ -693,15 +699,21 @@ bool scan_plan(int M, int d_v, int K, int in_bytes, ScanPlan* out)
     const int cols = ((Ml + 3) / 4) * cpl;
     uint32_t alloc = 32;
     while (alloc < static_cast<uint32_t>(cols)) alloc <<= 1;
-    const int S = 6, P = 2, X = 2;
-    int C = 64;
+    const int S = 6, X = 2;
+    int C = 64, P = 2;
     for (; C >= 1; C >>= 1) {
-        const int ft = (C + kFinWarps - 1) / kFinWarps;
-        if (ft * cpl > 8) continue;  // z values a finisher lane holds per chunk
+        const int ft = (C + kFinWarps / kFinGroups - 1) / (kFinWarps / kFinGroups);
+        if (ft * cpl > (cpl <= 4 ? 16 : 8)) continue;  // z values a finisher lane holds per chunk
         const size_t t = scan_layout(Ml, C, K, d_v, in_bytes, S, P, X, n, hdr_words_of(kScanWarps, C)).total;
         if (t <= static_cast<size_t>(kSmemBudget)) break;
     }
     if (C < 1) return false;
+    // a deeper read-partial ring, where it fits, lets the scan warps run further ahead of the
+    // finishers; the depth stays a multiple of kFinGroups, so every ring slot serves one
+    // finisher group and its barrier phases are consumed in order
+    if (scan_layout(Ml, C, K, d_v, in_bytes, S, 2 * P, X, n, hdr_words_of(kScanWarps, C)).total <=
+        static_cast<size_t>(kSmemBudget))
+        P *= 2;
     out->ncta = n;
     out->nw = kScanWarps;
     out->nfin = kFinWarps;
