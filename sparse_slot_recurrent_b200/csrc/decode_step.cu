@@ -280,11 +280,229 @@ cudaError_t step_k(const StepParams& p, cudaStream_t s)
     return launch_step<64, DPMAX>(p, s);
 }
 
+
+// ------------------------------------------------------------------ one warp per unit
+//
+// For K <= 16 and d_p <= 8 (the batched decode shapes) the step runs one warp per (b,h)
+// unit, with every unit of the batch resident at once (4 warps per CTA, up to 7 CTAs per
+// SM), so the address decode, the only long dependency chain of the step, takes one Top-K
+// search of latency and not a queue of them.
+//
+// Address decode: lanes 0-15 search the key (write) addresses, lanes 16-31 the query (read)
+// addresses, each 16-lane half on its own logits.  Lane i of a half holds the i-th best
+// prefix of the current level (the packed 64-bit candidate word of the prefix-tree search).
+// A level extends the kept prefixes by every digit: column j of the candidates is the kept
+// list shifted by digit code e[j] (codes sorted best first), so every column is sorted, and
+// the columns are merged pairwise by bitonic top-16 merges over warp shuffles (the element-
+// wise maximum of one list and the other reversed is bitonic and holds the 16 best; a
+// bitonic merge sorts it).  The kept words are distinct, so the 16 best, and the K best
+// among them, are unique: the result equals the one-thread search of the other kernels.
+// Then lane i computes winner i's weight, slot (after CAPE) and, for writes, retention.
+//
+// Rows: lane l owns channels [l*CPL, l*CPL + CPL) of every row; the K write rows are
+// loaded kStepRows at a time, updated by GSU step 4 and stored, then the K read rows are
+// loaded (a read row equal to a write row is the value this lane just stored: same address,
+// program order) and summed by weight; RMSNorm, norm weight, gate, y.
+
+constexpr int kWarpStepWarps = 4;
+
+// top-16 (best first) of two best-first 16-lists held one entry per lane of a 16-lane
+// segment; `b_rev` is the other list's entry at position 15 - li
+__device__ __forceinline__ uint64_t merge16(uint64_t a, uint64_t b_rev, int li)
+{
+    uint64_t x = a > b_rev ? a : b_rev;
+#pragma unroll
+    for (int d = 8; d > 0; d >>= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, x, d, 16);
+        x = (li & d) ? (x < y ? x : y) : (x > y ? x : y);
+    }
+    return x;
+}
+
+template <int DPMAX, int CPL>
+__global__ void __launch_bounds__(kWarpStepWarps * 32, 7) k_step_warp(StepParams p)
+{
+    constexpr int kStepRows = CPL >= 8 ? 4 : (CPL >= 4 ? 8 : 16);  // rows per lane in flight
+    const int lane = threadIdx.x & 31;
+    const int bh = static_cast<int>(blockIdx.x) * kWarpStepWarps + static_cast<int>(threadIdx.x >> 5);
+    if (bh >= p.B * p.H) return;  // whole warps only
+    const int half = lane >> 4, li = lane & 15;
+    const int K = p.K, dv = p.d_v, M = p.M, d_p = p.d_p, U = p.U;
+    const int L = U * d_p;
+    const void* lg = half == 0 ? p.k_logits : p.q_logits;
+    const size_t off = static_cast<size_t>(bh) * L;
+    const int h = bh % p.H, b = bh / p.H;
+
+    const int LW = (CPL > 1 || dv >= 32) ? 32 : dv;  // lanes holding channels
+    const bool act = lane < LW;
+    const int ch0 = (act ? lane : 0) * CPL;
+    prefetch_logits(lg, off, p.in_bf16, L);
+
+    // ---- exact Top-K by levels, one kept prefix per lane
+    uint64_t kept;
+    int nk;
+    {
+        uint64_t e[DPMAX];
+#pragma unroll
+        for (int d = 0; d < DPMAX; ++d)
+            e[d] = d < d_p ? digit_code(load_in(lg, off + d, p.in_bf16), d, d_p) : 0x8000000000000000ull;
+        sort_codes_desc<DPMAX>(e);
+        nk = min(K, d_p);
+        kept = 0ull;
+#pragma unroll
+        for (int d = 0; d < DPMAX; ++d)
+            if (d == li && d < nk) kept = (kKeyBias << 16) + e[d];
+    }
+    const uint64_t mul = static_cast<uint64_t>(d_p - 1);
+    for (int u = 1; u < U; ++u) {
+        uint64_t e[DPMAX];
+#pragma unroll
+        for (int d = 0; d < DPMAX; ++d)
+            e[d] = d < d_p ? digit_code(load_in(lg, off + u * d_p + d, p.in_bf16), d, d_p) : 0x8000000000000000ull;
+        sort_codes_desc<DPMAX>(e);
+        const uint64_t f = kept + (kept & 0xFFFFull) * mul;               // this lane's prefix, extended
+        const uint64_t fr = __shfl_sync(0xffffffffu, f, 15 - li, 16);   // the prefix at position 15 - li
+        const bool ok = li < nk, okr = 15 - li < nk;
+        uint64_t t[DPMAX / 2];
+#pragma unroll
+        for (int q = 0; q < DPMAX / 2; ++q) {
+            const uint64_t a = (ok && 2 * q < d_p) ? f + e[2 * q] : 0ull;
+            const uint64_t br = (okr && 2 * q + 1 < d_p) ? fr + e[2 * q + 1] : 0ull;
+            t[q] = merge16(a, br, li);
+        }
+#pragma unroll
+        for (int n = DPMAX / 2; n > 1; n >>= 1)
+#pragma unroll
+            for (int q = 0; q < n / 2; ++q)
+                t[q] = merge16(t[2 * q], __shfl_sync(0xffffffffu, t[2 * q + 1], 15 - li, 16), li);
+        nk = min(K, nk * d_p);
+        kept = li < nk ? t[0] : 0ull;  // only the K best prefixes are kept
+    }
+
+    // ---- winner li of this half: weight, slot after CAPE, retention (writes)
+    const bool win = li < K;
+    const int64_t s0 = packed_score(__shfl_sync(0xffffffffu, kept, 0, 16));
+    float base = 0.0f;
+    if (!p.renorm) {
+        float lse = 0.0f;
+        for (int uu = 0; uu < U; ++uu) {
+            float mx = -INFINITY;
+            for (int d = 0; d < d_p; ++d)
+                mx = fmaxf(mx, fminf(fmaxf(load_in(lg, off + uu * d_p + d, p.in_bf16), -4095.f), 4095.f));
+            float zs = 0.0f;
+            for (int d = 0; d < d_p; ++d)
+                zs += expf(fminf(fmaxf(load_in(lg, off + uu * d_p + d, p.in_bf16), -4095.f), 4095.f) - mx);
+            lse += mx + logf(zs);
+        }
+        base = static_cast<float>(s0) * kInvScale - lse;
+    }
+    float w = win ? expf(base + static_cast<float>(packed_score(kept) - s0) * kInvScale) : 0.0f;
+    if (p.renorm) {
+        float sum = w;
+#pragma unroll
+        for (int d = 8; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d, 16);
+        w = w / sum;
+    }
+    const bool cape = p.cape_mask != nullptr && p.cape_mask[h] != 0;
+    const int32_t pm = cape ? cape_shift(0, p.pos != nullptr ? p.pos[b] : 0, M) : 0;
+    int32_t idx = packed_index(kept, M) + pm;
+    if (idx >= M) idx -= M;
+    if (!dcheck(!win || (idx >= 0 && idx < M), p.status) || !win) idx = 0;
+
+    // ---- GSU steps 1-3 on the K write masses (lane j < K of the key half)
+    float* S = p.S + static_cast<size_t>(bh) * M * dv;
+    float* mrow = p.m + static_cast<size_t>(bh) * M;
+    float vv[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) vv[c] = act ? load_in(p.v, static_cast<size_t>(bh) * dv + ch0 + c, p.in_bf16) : 0.0f;
+    float lam = 0.0f;
+    if (half == 0 && win) {
+        const float gg = load_in(p.g, bh, p.in_bf16);
+        const float mn = gsu_alpha(w, gg) * mrow[idx] + w;
+        mrow[idx] = mn;
+        lam = w / (mn + p.eps_gsu);
+    }
+    // ---- GSU step 4 on the K write rows
+    for (int j0 = 0; j0 < K; j0 += kStepRows) {
+        float sr[kStepRows][CPL];
+        int ri[kStepRows];
+#pragma unroll
+        for (int k = 0; k < kStepRows; ++k) {
+            ri[k] = __shfl_sync(0xffffffffu, idx, (j0 + k) & 15);
+            if (j0 + k < K && act) load_row_g<CPL>(S + static_cast<size_t>(ri[k]) * dv + ch0, sr[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kStepRows; ++k) {
+            const float lk = __shfl_sync(0xffffffffu, lam, (j0 + k) & 15);
+            if (j0 + k < K && act) {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) sr[k][c] = fmaf(lk, vv[c] - sr[k][c], sr[k][c]);
+                store_row_g<CPL>(S + static_cast<size_t>(ri[k]) * dv + ch0, sr[k]);
+            }
+        }
+    }
+    // ---- read rows (after the writes), weighted sum
+    float o[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) o[c] = 0.0f;
+    for (int j0 = 0; j0 < K; j0 += kStepRows) {
+        float sr[kStepRows][CPL];
+#pragma unroll
+        for (int k = 0; k < kStepRows; ++k) {
+            const int rj = __shfl_sync(0xffffffffu, idx, 16 + ((j0 + k) & 15));
+            if (j0 + k < K && act) load_row_g<CPL>(S + static_cast<size_t>(rj) * dv + ch0, sr[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kStepRows; ++k) {
+            const float r = __shfl_sync(0xffffffffu, w, 16 + ((j0 + k) & 15));
+            if (j0 + k < K && act) {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) o[c] = fmaf(r, sr[k][c], o[c]);
+            }
+        }
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) ss = fmaf(o[c], o[c], ss);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, d);
+    const float inv = 1.0f / sqrtf(ss / dv + p.eps_norm);
+    if (act) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const float zc = load_in(p.z, static_cast<size_t>(bh) * dv + ch0 + c, p.in_bf16);
+            const float nc = p.norm_w != nullptr ? p.norm_w[ch0 + c] : 1.0f;
+            store_out(p.y, static_cast<size_t>(bh) * dv + ch0 + c, o[c] * inv * nc * zc, p.out_bf16);
+        }
+    }
+}
+
+template <int DPMAX>
+cudaError_t launch_step_warp(const StepParams& p, cudaStream_t s)
+{
+    const int units = p.B * p.H;
+    const unsigned grid = static_cast<unsigned>((units + kWarpStepWarps - 1) / kWarpStepWarps);
+    void (*kern)(StepParams) = nullptr;
+    switch (p.d_v < 32 ? 1 : p.d_v / 32) {
+        case 1: kern = k_step_warp<DPMAX, 1>; break;
+        case 2: kern = k_step_warp<DPMAX, 2>; break;
+        case 4: kern = k_step_warp<DPMAX, 4>; break;
+        case 8: kern = k_step_warp<DPMAX, 8>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    kern<<<grid, kWarpStepWarps * 32, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_decode_step(const StepParams& p, cudaStream_t stream)
 {
     if (p.d_v > 256) return cudaErrorInvalidValue;
+    // one warp per unit where the kept list fits a 16-lane half and a level's columns fit the
+    // merge tree; the persistent kernel otherwise
+    if (p.K <= 16 && p.d_p <= 4) return launch_step_warp<4>(p, stream);
+    if (p.K <= 16 && p.d_p <= 8) return launch_step_warp<8>(p, stream);
     if (p.d_p <= 4) return step_k<4>(p, stream);
     if (p.d_p <= 8) return step_k<8>(p, stream);
     return step_k<16>(p, stream);
