@@ -598,6 +598,48 @@ def test_decode_step_matches_oracle_over_steps():
     assert _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
 
 
+STEP_SEARCH_CASES = [
+    # d_p, U, K, logit mode, renorm -- shapes of the one-warp-per-unit step (K <= 16, d_p <= 8)
+    (8, 4, 16, "ties", 1),
+    (8, 4, 16, "mixed", 0),
+    (4, 5, 8, "ties", 1),
+    (3, 4, 5, "mixed", 1),
+    (2, 8, 16, "ties", 0),
+    (8, 2, 1, "normal", 1),
+    (5, 3, 12, "ties", 1),
+]
+
+
+@pytest.mark.parametrize("d_p,U,K,mode,renorm", STEP_SEARCH_CASES)
+def test_decode_step_cooperative_search_matches_oracle(d_p, U, K, mode, renorm):
+    """Decode steps whose Top-K runs on 16-lane halves of a warp, with tie-heavy and mixed
+    logits: a slot chosen wrongly among equal scores writes a different row of S."""
+    B, H, steps, d_v = 3, 5, 3, 32
+    cfg = ramnet.Config(d_p=d_p, U=U, K=K, d_v=d_v, renorm=renorm)
+    ocfg = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=d_v, renorm=renorm)
+    M = d_p ** U
+    g = torch.Generator().manual_seed(d_p * 1000 + K)
+    S0 = torch.randn((B, H, M, d_v), generator=g)
+    m0 = torch.rand((B, H, M), generator=g) + 0.5
+    S, m = S0.cuda(), m0.cuda()
+    oS, om = S0.double().numpy().copy(), m0.double().numpy().copy()
+    mask = torch.tensor([1, 0, 1, 1, 0], dtype=torch.uint8)
+    kl = _logits(B, steps, H, d_p * U, mode, torch.float32, seed=K + 1)
+    ql = _logits(B, steps, H, d_p * U, mode, torch.float32, seed=K + 2)
+    for t in range(steps):
+        v = torch.randn((B, H, d_v), generator=g)
+        z = torch.sigmoid(torch.randn((B, H, d_v), generator=g))
+        gt = torch.sigmoid(torch.randn((B, H), generator=g))
+        pos = torch.tensor([t, 77 + t, M + 5 + t], dtype=torch.int32)
+        k_t, q_t = kl[:, t].contiguous(), ql[:, t].contiguous()
+        y = ramnet.decode_step(cfg, k_t.cuda(), q_t.cuda(), v.cuda(), gt.cuda(), z.cuda(), S, m, pos=pos.cuda(),
+                               cape_mask=mask.cuda(), out_dtype=torch.float32)
+        oy = oracle.decode_step(ocfg, k_t, q_t, v, gt, z, oS, om, pos=pos, cape_mask=mask)
+        ramnet.sync_status()
+        assert _maxabs(y, oy) <= TOL_F32
+    assert _maxabs(S, oS) <= TOL_F32 and _maxabs(m, om) <= TOL_F32
+
+
 def test_decode_step_full_size_sampled_units():
     """One step of the full batched decode workload (state resident in HBM); sampled
     (b,h) units are recomputed by the oracle from their pre-step state."""
