@@ -442,7 +442,9 @@ def run_gpu(args, world, rank, local):
             print(json.dumps({"metric": METRIC, "decode": decode}), flush=True)
         return
     head = WORKLOADS[args.workload]
-    others = [] if args.only_headline else [n for n in PREFILL_ALL if n != head.name]
+    if args.prefill_batch:  # fewer sequences of the same layer (profiler captures); headline only
+        head = head.with_(B=args.prefill_batch, name=f"{head.name}_b{args.prefill_batch}")
+    others = [] if (args.only_headline or args.prefill_batch) else [n for n in PREFILL_ALL if n != head.name]
     main = time_prefill(args, world, rank, local, head, with_e2e=not args.no_e2e)
     prefill = {head.name: {k: v for k, v in main.items() if k != "e2e"}}
     for name in others:
@@ -531,6 +533,9 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[k for k, v in WORKLOADS.items() if not v.decode],
                     help="headline prefill workload (default: the 1.3B-like Top-16 long-context layer)")
     ap.add_argument("--only-headline", action="store_true", help="time only the headline prefill workload")
+    ap.add_argument("--prefill-batch", type=int, default=0,
+                    help="sequences of the headline prefill workload (default: the workload's; smaller for profiler "
+                         "captures, timed as that workload only)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences of the decode workload (default 256; smaller for profiler captures)")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill workloads (decode only)")
