@@ -338,15 +338,59 @@ __global__ void __launch_bounds__(kWarpStepWarps * 32, 7) k_step_warp(StepParams
     const int ch0 = (act ? lane : 0) * CPL;
     prefetch_logits(lg, off, p.in_bf16, L);
 
+    // ---- digit codes, computed once per half: in a round, lane li of a half takes digit
+    // li mod DPMAX of level (round * LPR + li / DPMAX); each level's DPMAX lanes sort their
+    // codes best first (bitonic, by signed value as sort_codes_desc) and, for the raw product
+    // softmax, reduce the level's logsumexp.  A level's sorted codes reach every lane of the
+    // half by shuffles.
+    constexpr int LPR = 16 / DPMAX;  // levels per round
+    const int dpos = li % DPMAX, dseg = (li / DPMAX) * DPMAX;
+    uint64_t cs = 0ull;  // this lane's sorted code of its level in the current round
+    float lse = 0.0f;    // sum over levels of logsumexp (renorm == 0)
+    auto code_round = [&](int r) {
+        const int u = r * LPR + li / DPMAX;
+        const bool valid = u < U && dpos < d_p;
+        const float x = valid ? load_in(lg, off + u * d_p + dpos, p.in_bf16) : 0.0f;
+        uint64_t c = valid ? digit_code(x, dpos, d_p) : 0x8000000000000000ull;
+#pragma unroll
+        for (int k = 2; k <= DPMAX; k <<= 1)
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                const int64_t o = static_cast<int64_t>(__shfl_xor_sync(0xffffffffu, c, j, 16));
+                const int64_t v = static_cast<int64_t>(c);
+                const bool keep_max = ((dpos & j) == 0) == ((dpos & k) == 0);
+                c = static_cast<uint64_t>(keep_max ? (v > o ? v : o) : (v < o ? v : o));
+            }
+        cs = c;
+        if (!p.renorm) {
+            const float xc = fminf(fmaxf(x, -4095.f), 4095.f);
+            float mx = valid ? xc : -INFINITY;
+#pragma unroll
+            for (int j = DPMAX / 2; j > 0; j >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, j, 16));
+            float zs = valid ? expf(xc - mx) : 0.0f;
+#pragma unroll
+            for (int j = DPMAX / 2; j > 0; j >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, j, 16);
+            float l = (u < U) ? mx + logf(zs) : 0.0f;  // this level's logsumexp (every lane of the level)
+            // add the round's levels: one value per DPMAX-lane segment of the half
+            float acc = l;
+#pragma unroll
+            for (int j = DPMAX; j < 16; j <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, j, 16);
+            lse += acc;
+        }
+    };
+    auto level_codes = [&](int u, uint64_t (&e)[DPMAX]) {
+        if (u % LPR == 0) code_round(u / LPR);
+        const int base = (u % LPR) * DPMAX;
+#pragma unroll
+        for (int d = 0; d < DPMAX; ++d) e[d] = __shfl_sync(0xffffffffu, cs, base + d, 16);
+    };
+
     // ---- exact Top-K by levels, one kept prefix per lane
     uint64_t kept;
     int nk;
     {
         uint64_t e[DPMAX];
-#pragma unroll
-        for (int d = 0; d < DPMAX; ++d)
-            e[d] = d < d_p ? digit_code(load_in(lg, off + d, p.in_bf16), d, d_p) : 0x8000000000000000ull;
-        sort_codes_desc<DPMAX>(e);
+        level_codes(0, e);
         nk = min(K, d_p);
         kept = 0ull;
 #pragma unroll
@@ -356,10 +400,7 @@ __global__ void __launch_bounds__(kWarpStepWarps * 32, 7) k_step_warp(StepParams
     const uint64_t mul = static_cast<uint64_t>(d_p - 1);
     for (int u = 1; u < U; ++u) {
         uint64_t e[DPMAX];
-#pragma unroll
-        for (int d = 0; d < DPMAX; ++d)
-            e[d] = d < d_p ? digit_code(load_in(lg, off + u * d_p + d, p.in_bf16), d, d_p) : 0x8000000000000000ull;
-        sort_codes_desc<DPMAX>(e);
+        level_codes(u, e);
         const uint64_t f = kept + (kept & 0xFFFFull) * mul;               // this lane's prefix, extended
         const uint64_t fr = __shfl_sync(0xffffffffu, f, 15 - li, 16);   // the prefix at position 15 - li
         const bool ok = li < nk, okr = 15 - li < nk;
@@ -378,24 +419,12 @@ __global__ void __launch_bounds__(kWarpStepWarps * 32, 7) k_step_warp(StepParams
         nk = min(K, nk * d_p);
         kept = li < nk ? t[0] : 0ull;  // only the K best prefixes are kept
     }
+    // (every round of levels 0..U-1 was reached above, so lse covers all U levels)
 
     // ---- winner li of this half: weight, slot after CAPE, retention (writes)
     const bool win = li < K;
     const int64_t s0 = packed_score(__shfl_sync(0xffffffffu, kept, 0, 16));
-    float base = 0.0f;
-    if (!p.renorm) {
-        float lse = 0.0f;
-        for (int uu = 0; uu < U; ++uu) {
-            float mx = -INFINITY;
-            for (int d = 0; d < d_p; ++d)
-                mx = fmaxf(mx, fminf(fmaxf(load_in(lg, off + uu * d_p + d, p.in_bf16), -4095.f), 4095.f));
-            float zs = 0.0f;
-            for (int d = 0; d < d_p; ++d)
-                zs += expf(fminf(fmaxf(load_in(lg, off + uu * d_p + d, p.in_bf16), -4095.f), 4095.f) - mx);
-            lse += mx + logf(zs);
-        }
-        base = static_cast<float>(s0) * kInvScale - lse;
-    }
+    const float base = p.renorm ? 0.0f : static_cast<float>(s0) * kInvScale - lse;
     float w = win ? expf(base + static_cast<float>(packed_score(kept) - s0) * kInvScale) : 0.0f;
     if (p.renorm) {
         float sum = w;
