@@ -274,6 +274,19 @@ ramnet_status ramnet_decode_step(const ramnet_config* cfg, int32_t B, int32_t H,
 ramnet_status ramnet_selftest_wait_timeout(uint32_t limit_us, void* stream);
 
 /*
+ * ramnet_set_scan_wait_limit -- failure-detection hook, no counterpart in the pages.  Sets
+ * the limit of every bounded wait inside the prefill recurrence (ramnet_scan_recur,
+ * ramnet_scan_forward, ramnet_scan_forward_noalloc) launched after the call, for the whole
+ * process: limit_us microseconds, or 0 for the default of 2 s.  A wait that runs out records
+ * RAMNET_ERR_TIMEOUT in the device status word and the kernel winds down: its remaining
+ * work is skipped, so y, S_out and m_out are then incomplete.  A limit far below the
+ * kernel's own hand-over times makes the recurrence time out on purpose, which is how its
+ * abort path is tested.
+ * Errors: INVALID_ARG if limit_us > 2000000.
+ */
+ramnet_status ramnet_set_scan_wait_limit(uint32_t limit_us);
+
+/*
  * ramnet_sync_status -- waits for `stream`, then returns RAMNET_ERR_TIMEOUT or
  * RAMNET_ERR_DEVICE_CHECK if a kernel of this library on the current device recorded a
  * gave-up wait or a failed check since the last call (and clears the record), or

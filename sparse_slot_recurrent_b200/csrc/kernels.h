@@ -92,6 +92,7 @@ struct ScanParams {
     int ncta, nw, nfin, chunk, nch, stages, lslots, xslots, hdr_words;
     float eps_gsu, eps_norm;
     uint32_t tmem_cols;
+    uint64_t wait_ns;  // limit of every bounded wait of the kernel
     uint32_t* status;
 };
 

@@ -1,5 +1,6 @@
 // ramnet_api.cu -- the C ABI declared in include/ramnet.h: argument checks, launches,
 // status reporting.  Nothing here allocates device memory.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <string>
@@ -10,6 +11,8 @@
 namespace {
 
 thread_local std::string g_last_error;
+// limit of every bounded wait of the prefill recurrence (process-wide; ramnet_set_scan_wait_limit)
+std::atomic<uint64_t> g_scan_wait_ns{2000000000ull};
 
 // Device-side status word of this library (one per device that loads the library).
 __device__ uint32_t g_device_status;
@@ -267,6 +270,7 @@ ramnet_status recur_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
     sp.eps_gsu = cfg->eps_gsu;
     sp.eps_norm = cfg->eps_norm;
     sp.tmem_cols = plan.tmem_cols;
+    sp.wait_ns = g_scan_wait_ns.load(std::memory_order_relaxed);
     sp.status = status;
     cudaError_t e = ramnet::launch_scan(sp, plan.smem_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
@@ -362,6 +366,15 @@ ramnet_status ramnet_selftest_wait_timeout(uint32_t limit_us, void* stream)
     cudaError_t e = ramnet::launch_wait_selftest(status, static_cast<uint64_t>(limit_us) * 1000ull,
                                                  static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+    return RAMNET_OK;
+}
+
+ramnet_status ramnet_set_scan_wait_limit(uint32_t limit_us)
+{
+    g_last_error.clear();
+    if (limit_us > 2000000) return fail(RAMNET_ERR_INVALID_ARG, "limit_us=%u above 2000000", limit_us);
+    g_scan_wait_ns.store(limit_us == 0 ? 2000000000ull : static_cast<uint64_t>(limit_us) * 1000ull,
+                         std::memory_order_relaxed);
     return RAMNET_OK;
 }
 

@@ -106,13 +106,13 @@ __device__ __forceinline__ uint64_t global_ns()
 }
 
 // One try_wait on phase `parity`: the thread may be suspended in hardware until the phase
-// completes or about kSuspendNs have passed.  CLUSTER selects acquire at cluster scope (for
+// completes or about `hint_ns` (at most kSuspendNs) have passed.  CLUSTER selects acquire at cluster scope (for
 // barriers that peers of the cluster arrive on after writing into this CTA's shared memory);
 // otherwise the default CTA scope.
 constexpr uint32_t kSuspendNs = 100000;
 
 template <bool CLUSTER>
-__device__ __forceinline__ bool try_wait_phase(uint32_t bar, uint32_t parity)
+__device__ __forceinline__ bool try_wait_phase(uint32_t bar, uint32_t parity, uint32_t hint_ns = kSuspendNs)
 {
     uint32_t ok;
     if constexpr (CLUSTER) {
@@ -121,7 +121,7 @@ __device__ __forceinline__ bool try_wait_phase(uint32_t bar, uint32_t parity)
             "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity), "r"(kSuspendNs)
+            : "r"(bar), "r"(parity), "r"(hint_ns)
             : "memory");
     } else {
         asm volatile(
@@ -129,14 +129,15 @@ __device__ __forceinline__ bool try_wait_phase(uint32_t bar, uint32_t parity)
             "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity), "r"(kSuspendNs)
+            : "r"(bar), "r"(parity), "r"(hint_ns)
             : "memory");
     }
     return ok != 0;
 }
 
 // Bounded wait for phase `parity` of the mbarrier at shared address `bar`: at most
-// kSpinLimit polls and `limit_ns` (2 s unless given).  Between polls the thread sleeps
+// kSpinLimit polls and `limit_ns` (2 s unless given; the prefill recurrence passes its
+// launch's limit).  Between polls the thread sleeps
 // (32 ns doubling to 256 ns), so waiting warps leave the issue slots to working ones.  On
 // expiry the status word gets kDevTimeout and the CTA's abort flag is raised, after which
 // every later wait of the CTA returns at once, so a kernel that lost a signal still ends
@@ -145,12 +146,14 @@ template <bool CLUSTER>
 __device__ __forceinline__ void wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status, volatile int* abort_flag,
                                              uint64_t limit_ns = 2000000000ull)
 {
-    if (try_wait_phase<CLUSTER>(bar, parity)) return;
+    // a hardware suspension never outlasts the limit itself
+    const uint32_t hint = limit_ns < kSuspendNs ? static_cast<uint32_t>(limit_ns) : kSuspendNs;
+    if (try_wait_phase<CLUSTER>(bar, parity, hint)) return;
     if (*abort_flag) return;
     const uint64_t t_end = global_ns() + limit_ns;
     uint32_t nap = 32;
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
-        if (try_wait_phase<CLUSTER>(bar, parity)) return;
+        if (try_wait_phase<CLUSTER>(bar, parity, hint)) return;
         if (global_ns() > t_end || *abort_flag) break;
         __nanosleep(nap);
         nap = nap < 256 ? 2 * nap : 256;
@@ -379,9 +382,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
         tmem_wait_st();
         const unsigned lt_mask = (1u << lane) - 1u;
         for (int c = 0; c < nch; ++c) {
-            wait_bounded<false>(bar(BI.sfull + c % S), (c / S) & 1, p.status, abort_flag);
+            wait_bounded<false>(bar(BI.sfull + c % S), (c / S) & 1, p.status, abort_flag, p.wait_ns);
             const int ls = c % P, kl = c / P;
-            if (kl >= 1) wait_bounded<false>(bar(BI.lfree + ls), (kl - 1) & 1, p.status, abort_flag);
+            if (kl >= 1) wait_bounded<false>(bar(BI.lfree + ls), (kl - 1) & 1, p.status, abort_flag, p.wait_ns);
             const unsigned char* st = stage(c);
             const uint32_t* hd = reinterpret_cast<const uint32_t*>(st);
             if (!*abort_flag) {
@@ -521,7 +524,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
                     }
                 }
             }
-            wait_bounded<false>(bar(BI.ldone + ls), kl & 1, p.status, abort_flag);
+            wait_bounded<false>(bar(BI.ldone + ls), kl & 1, p.status, abort_flag, p.wait_ns);
             // this CTA's sum of each token's read partials, in q order
             const float* lr = lring + static_cast<size_t>(ls) * lslot_floats + lch;
             float o[kZMax];
@@ -545,8 +548,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             __syncwarp();
             if (lane == 0) arrive_local(bar(BI.lfree + ls));
             if (ncta > 1) {
-                if (own) wait_bounded<true>(bar(BI.xfull + xs), kx & 1, p.status, abort_flag);
-                else if (kx >= 1) wait_bounded<true>(bar(BI.xfree + f * X + xs), (kx - 1) & 1, p.status, abort_flag);
+                if (own) wait_bounded<true>(bar(BI.xfull + xs), kx & 1, p.status, abort_flag, p.wait_ns);
+                else if (kx >= 1) wait_bounded<true>(bar(BI.xfree + f * X + xs), (kx - 1) & 1, p.status, abort_flag, p.wait_ns);
             }
             const int xi = rank < f ? rank : rank - 1;  // this CTA's entry in f's exchange slot
             const uint32_t xdst = ncta > 1 && !own
@@ -633,7 +636,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan(ScanParams p)
             const uint32_t first = min(start, static_cast<uint32_t>(cap) - n);
             const int nt = min(C, p.T - c * C);
             if (c >= S) {
-                wait_bounded<false>(bar(BI.sfree + c % S), (c / S - 1) & 1, p.status, abort_flag);
+                wait_bounded<false>(bar(BI.sfree + c % S), (c / S - 1) & 1, p.status, abort_flag, p.wait_ns);
                 fence_proxy_async();
             }
             if (*abort_flag) continue;

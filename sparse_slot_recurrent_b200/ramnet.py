@@ -25,7 +25,7 @@ RAMNET_F32, RAMNET_BF16 = 0, 1
 # every symbol include/ramnet.h declares
 EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_layout", "ramnet_scan_forward",
             "ramnet_scan_route", "ramnet_scan_recur", "ramnet_scan_forward_noalloc", "ramnet_decode_step",
-            "ramnet_selftest_wait_timeout", "ramnet_sync_status", "ramnet_last_error")
+            "ramnet_selftest_wait_timeout", "ramnet_set_scan_wait_limit", "ramnet_sync_status", "ramnet_last_error")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # RAMNET_NOALLOC_SCRATCH_BYTES
 
 
@@ -108,6 +108,8 @@ def load() -> ctypes.CDLL:
                                        ctypes.c_int, _P]
     lib.ramnet_selftest_wait_timeout.restype = ctypes.c_int
     lib.ramnet_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
+    lib.ramnet_set_scan_wait_limit.restype = ctypes.c_int
+    lib.ramnet_set_scan_wait_limit.argtypes = [ctypes.c_uint32]
     lib.ramnet_sync_status.restype = ctypes.c_int
     lib.ramnet_sync_status.argtypes = [_P]
     lib.ramnet_last_error.restype = ctypes.c_char_p
@@ -271,6 +273,11 @@ def decode_step(cfg: Config, k_logits, q_logits, v, g, z, S, m, pos=None, norm_w
 def selftest_wait_timeout(limit_us: int, stream=None):
     """Launch the failure-detection self-test (a bounded wait that must run out)."""
     _check(load().ramnet_selftest_wait_timeout(limit_us, _stream(stream)))
+
+
+def set_scan_wait_limit(limit_us: int):
+    """Limit of the prefill recurrence's bounded waits for later launches (0: 2 s default)."""
+    _check(load().ramnet_set_scan_wait_limit(limit_us))
 
 
 def sync_status(stream=None):
