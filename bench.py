@@ -50,6 +50,7 @@ from sparse_slot_recurrent_b200.workloads import WORKLOADS, generate  # noqa: E4
 METRIC = "RAM-Net layer tokens/s (prefill scan, decode step) and % of HBM roofline"
 # the largest prefill configuration is the headline; the other two are timed beside it
 PREFILL = "prefill_1p3b_top16"
+E2E_PIECES = 8  # runs along T of the end-to-end call (copies of one run overlap another's kernels)
 PREFILL_ALL = ("prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16")
 LAUNCHES_PER_STEP = 2  # route (k_route) and recurrence (k_scan)
 SM_COUNT = 148
@@ -396,19 +397,22 @@ def time_prefill(args, world, rank, local, w, with_e2e: bool):
                  "frac": alg / (ms / 1e3) / 1e9 / peak},
     }
 
-    # end to end through the public API from pinned host memory
+    # end to end through the public API from pinned host memory: ramnet_scan_forward_host reads
+    # the step's per-token inputs from the host and writes y back to the host, in E2E_PIECES runs
+    # along T whose copies overlap the kernels
     e2e = None
     if with_e2e:
-        keys = ("k_logits", "q_logits", "v", "g", "z", "cape_mask", "pos0")
+        keys = ("k_logits", "q_logits", "v", "g", "z")
         yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
         h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
         d2h = yh.numel() * yh.element_size()
+        scratch = torch.empty(ramnet.scan_forward_host_scratch_bytes(cfg, w.B, w.T, w.H, w.in_dtype, out_dtype,
+                                                                     E2E_PIECES), dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            for k in keys:
-                d[k].copy_(host[k], non_blocking=True)
-            step()
-            yh.copy_(y, non_blocking=True)
+            ramnet.scan_forward_host(cfg, host["k_logits"], host["q_logits"], host["v"], host["g"], host["z"], yh, S, m,
+                                     scratch, pieces=E2E_PIECES, cape_mask=d["cape_mask"], pos0=d["pos0"],
+                                     stream=stream)
 
         for _ in range(2):
             e2e_step()
@@ -422,9 +426,12 @@ def time_prefill(args, world, rank, local, w, with_e2e: bool):
             e2e_step()
             ee[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        ramnet.sync_status(stream)
         e_ms = dist_max(statistics.mean(a.elapsed_time(b) for a, b in ee), world)
         e2e = {"value": weak_scaling_value(tokens, world, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": n_e2e}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": n_e2e, "pieces": E2E_PIECES,
+               "call": "ramnet_scan_forward_host"}
+        del scratch
     del flush, ws, y, S, m, d
     torch.cuda.empty_cache()
     return {"workload": w.name, "config": config_of(w, world), "value": value, "unit": "tokens/s",

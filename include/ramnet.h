@@ -209,6 +209,39 @@ ramnet_status ramnet_scan_recur(const ramnet_config* cfg, int32_t B, int32_t T, 
                                 ramnet_dtype out_dt, float* S_out, float* m_out,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * ramnet_scan_forward_host -- the prefill scan with the per-token tensors in HOST memory:
+ * k_logits, q_logits, v, g, z ([B,T,H,.], last dim contiguous, as ramnet_scan_forward) are
+ * read from the host and y is written to the host; norm_w, cape_mask, pos0, S_in, m_in,
+ * S_out and m_out are device pointers as in ramnet_scan_forward.  Same results as
+ * ramnet_scan_forward, bit for bit.
+ *
+ * The sequence is cut into `pieces` runs of ceil(T / pieces) tokens.  The scan is causal
+ * and its state (S, m) is the whole carry, so run i starts from the state run i-1 left in
+ * S_out / m_out (run 0 from S_in / m_in) and its CAPE positions continue at
+ * pos0[b] + (first token of the run); this is the RAM-Net project page's recurrence taken
+ * piece by piece.  Copies of run i+1 into the device and of run i-1's y out of it overlap
+ * run i's kernels (two copy streams created for the call; page-locked host memory lets the
+ * copies run asynchronously).  Work is ordered after earlier work on `stream`, and
+ * `stream` waits for the whole call, the last copy out included.
+ *
+ *   scratch: device memory of ramnet_scan_forward_host_scratch_bytes() bytes (two
+ *            staging buffers for the inputs and y of a run, and one workspace), 16-byte
+ *            aligned, owned by the caller and not used by other work during the call.
+ *   Errors:  INVALID_ARG (NULL host tensor, pieces < 1, scratch too small, and the checks
+ *            of ramnet_scan_forward), UNSUPPORTED, CUDA.
+ */
+size_t ramnet_scan_forward_host_scratch_bytes(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                              ramnet_dtype in_dt, ramnet_dtype out_dt, int32_t pieces);
+ramnet_status ramnet_scan_forward_host(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                       ramnet_dtype in_dt, const void* k_logits, const void* q_logits,
+                                       const void* v, const void* g, const void* z,
+                                       const float* norm_w, const uint8_t* cape_mask,
+                                       const int32_t* pos0, const float* S_in, const float* m_in,
+                                       void* y, ramnet_dtype out_dt, float* S_out, float* m_out,
+                                       int32_t pieces, void* scratch, size_t scratch_bytes,
+                                       void* stream);
+
 /* Size of the scratch array built into the library for ramnet_scan_forward_noalloc. */
 #define RAMNET_NOALLOC_SCRATCH_BYTES ((size_t)32 * 1024 * 1024)
 

@@ -68,6 +68,7 @@ struct RouteParams {
     int d_p, U, K, M, renorm;
     int B, T, H;
     const int32_t* pos0;       // [B] or null
+    int64_t t_offset;          // position of token 0 relative to pos0 (pieces of a longer sequence)
     const uint8_t* cape_mask;  // [H] or null
     int ncta, nw, chunk, nch, hdr_words;
     uint4* events;

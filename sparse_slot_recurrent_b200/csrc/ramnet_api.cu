@@ -201,9 +201,10 @@ ramnet_status check_scan(const ramnet_config* cfg, int32_t B, int32_t T, int32_t
 ramnet_status route_part(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt, int M,
                          const ramnet::ScanPlan& plan, const ramnet::ScanWorkspace& wl, const void* k_logits,
                          const void* q_logits, const void* g, const uint8_t* cape_mask, const int32_t* pos0,
-                         void* workspace, cudaStream_t s)
+                         void* workspace, cudaStream_t s, int64_t t_offset = 0)
 {
     ramnet::RouteParams rp{};
+    rp.t_offset = t_offset;
     rp.k_logits = k_logits;
     rp.q_logits = q_logits;
     rp.g = g;
@@ -446,6 +447,181 @@ ramnet_status ramnet_sync_status(void* stream)
         if (word & ramnet::kDevTimeout) return fail(RAMNET_ERR_TIMEOUT, "a device-side wait gave up (status 0x%x)", word);
         return fail(RAMNET_ERR_DEVICE_CHECK, "a device-side check failed (status 0x%x)", word);
     }
+    return RAMNET_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ prefill from host memory
+namespace {
+
+struct HostPieces {
+    int n;          // pieces
+    int tp;         // tokens per piece (the last may be shorter)
+    size_t in_piece[5];  // bytes of one piece of k, q, v, g, z
+    size_t y_piece;
+    size_t in_off[2][5], y_off[2], ws_off, total;
+    ramnet::ScanWorkspace wl;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+HostPieces host_pieces(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                       ramnet_dtype out_dt, int32_t pieces, const ramnet::ScanPlan& plan)
+{
+    HostPieces hp{};
+    hp.n = pieces < 1 ? 1 : (pieces > T ? T : pieces);
+    hp.tp = (T + hp.n - 1) / hp.n;
+    hp.n = (T + hp.tp - 1) / hp.tp;
+    const size_t es = in_dt == RAMNET_BF16 ? 2 : 4, eo = out_dt == RAMNET_BF16 ? 2 : 4;
+    const size_t th = static_cast<size_t>(B) * hp.tp * H;
+    const size_t L = static_cast<size_t>(cfg->U) * cfg->d_p;
+    hp.in_piece[0] = hp.in_piece[1] = th * L * es;
+    hp.in_piece[2] = hp.in_piece[4] = th * cfg->d_v * es;
+    hp.in_piece[3] = th * es;
+    hp.y_piece = th * cfg->d_v * eo;
+    size_t o = 0;
+    for (int buf = 0; buf < 2; ++buf) {
+        for (int i = 0; i < 5; ++i) {
+            hp.in_off[buf][i] = o;
+            o += align256(hp.in_piece[i]);
+        }
+        hp.y_off[buf] = o;
+        o += align256(hp.y_piece);
+    }
+    hp.wl = ramnet::scan_workspace(B, hp.tp, H, cfg->K, plan);
+    hp.ws_off = o;
+    o += align256(hp.wl.total);
+    hp.total = o;
+    return hp;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ramnet_scan_forward_host_scratch_bytes(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H,
+                                              ramnet_dtype in_dt, ramnet_dtype out_dt, int32_t pieces)
+{
+    g_last_error.clear();
+    int M = 0;
+    if (check_config(cfg, &M) != RAMNET_OK || check_sizes(B, T, H) != RAMNET_OK || !valid_dtype(in_dt) ||
+        !valid_dtype(out_dt))
+        return 0;
+    ramnet::ScanPlan plan;
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, &plan)) return 0;
+    return host_pieces(cfg, B, T, H, in_dt, out_dt, pieces, plan).total;
+}
+
+ramnet_status ramnet_scan_forward_host(const ramnet_config* cfg, int32_t B, int32_t T, int32_t H, ramnet_dtype in_dt,
+                                       const void* k_logits, const void* q_logits, const void* v, const void* g,
+                                       const void* z, const float* norm_w, const uint8_t* cape_mask,
+                                       const int32_t* pos0, const float* S_in, const float* m_in, void* y,
+                                       ramnet_dtype out_dt, float* S_out, float* m_out, int32_t pieces,
+                                       void* scratch, size_t scratch_bytes, void* stream)
+{
+    g_last_error.clear();
+    int M = 0;
+    ramnet_status st = check_config(cfg, &M);
+    if (st != RAMNET_OK) return st;
+    if ((st = check_sizes(B, T, H)) != RAMNET_OK) return st;
+    if (!valid_dtype(in_dt) || !valid_dtype(out_dt)) return fail(RAMNET_ERR_INVALID_ARG, "bad dtype");
+    if (pieces < 1) return fail(RAMNET_ERR_INVALID_ARG, "pieces=%d < 1", pieces);
+    if (k_logits == nullptr || q_logits == nullptr || v == nullptr || g == nullptr || z == nullptr || y == nullptr)
+        return fail(RAMNET_ERR_INVALID_ARG, "a host input or y is NULL");
+    REQUIRE_PTR(S_out);
+    REQUIRE_PTR(m_out);
+    REQUIRE_PTR(scratch);
+    OPTIONAL_PTR(norm_w);
+    OPTIONAL_PTR(cape_mask);
+    OPTIONAL_PTR(pos0);
+    OPTIONAL_PTR(S_in);
+    OPTIONAL_PTR(m_in);
+    ramnet::ScanPlan plan;
+    if (!ramnet::scan_plan(M, cfg->d_v, cfg->K, in_dt == RAMNET_BF16 ? 2 : 4, &plan))
+        return fail(RAMNET_ERR_UNSUPPORTED, "slot array M=%d x d_v=%d does not fit the tensor memory of 8 SMs", M,
+                    cfg->d_v);
+    const HostPieces hp = host_pieces(cfg, B, T, H, in_dt, out_dt, pieces, plan);
+    if (scratch_bytes < hp.total)
+        return fail(RAMNET_ERR_INVALID_ARG, "scratch of %zu bytes, %zu needed", scratch_bytes, hp.total);
+
+    const size_t es = in_dt == RAMNET_BF16 ? 2 : 4, eo = out_dt == RAMNET_BF16 ? 2 : 4;
+    const size_t L = static_cast<size_t>(cfg->U) * cfg->d_p;
+    const size_t row_bytes[5] = {L * es, L * es, static_cast<size_t>(cfg->d_v) * es, es,
+                                 static_cast<size_t>(cfg->d_v) * es};  // per token-head
+    const void* src[5] = {k_logits, q_logits, v, g, z};
+    unsigned char* base = static_cast<unsigned char*>(scratch);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // copy-in and copy-out streams; events order them against the compute stream `s`
+    cudaStream_t sin = nullptr, sout = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_in[2] = {nullptr, nullptr}, ev_done[2] = {nullptr, nullptr},
+                ev_out[2] = {nullptr, nullptr};
+    cudaError_t e = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+        e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming);
+    }
+    // the staging buffers may still be in use by earlier work on `s`
+    if (e == cudaSuccess) e = cudaEventRecord(ev_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sin, ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, ev_start, 0);
+    for (int i = 0; i < hp.n && e == cudaSuccess && st == RAMNET_OK; ++i) {
+        const int buf = i & 1;
+        const int t0 = i * hp.tp, tn = (T - t0) < hp.tp ? (T - t0) : hp.tp;
+        // inputs of piece i: B rows of tn*H token-heads each, strided by T*H in the host arrays
+        if (i >= 2) e = cudaStreamWaitEvent(sin, ev_done[buf], 0);  // piece i-2 consumed its inputs
+        for (int a = 0; a < 5 && e == cudaSuccess; ++a) {
+            const size_t w = static_cast<size_t>(tn) * H * row_bytes[a];
+            e = cudaMemcpy2DAsync(base + hp.in_off[buf][a], w, static_cast<const unsigned char*>(src[a]) +
+                                  static_cast<size_t>(t0) * H * row_bytes[a],
+                                  static_cast<size_t>(T) * H * row_bytes[a], w, static_cast<size_t>(B),
+                                  cudaMemcpyHostToDevice, sin);
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[buf], sin);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in[buf], 0);
+        if (e == cudaSuccess && i >= 2) e = cudaStreamWaitEvent(s, ev_out[buf], 0);  // y staging of piece i-2 read
+        if (e != cudaSuccess) break;
+        // piece i on the compute stream; the state is carried in S_out / m_out
+        void* ws = base + hp.ws_off;
+        const float* Si = i == 0 ? S_in : S_out;
+        const float* mi = i == 0 ? m_in : m_out;
+        const ramnet::ScanWorkspace wl = ramnet::scan_workspace(B, tn, H, cfg->K, plan);
+        st = route_part(cfg, B, tn, H, in_dt, M, plan, wl, base + hp.in_off[buf][0], base + hp.in_off[buf][1],
+                        base + hp.in_off[buf][3], cape_mask, pos0, ws, s, t0);
+        if (st == RAMNET_OK)
+            st = recur_part(cfg, B, tn, H, in_dt, M, plan, wl, base + hp.in_off[buf][2], base + hp.in_off[buf][4],
+                            norm_w, Si, mi, base + hp.y_off[buf], out_dt, S_out, m_out, ws, s);
+        if (st != RAMNET_OK) break;
+        e = cudaEventRecord(ev_done[buf], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, ev_done[buf], 0);
+        if (e == cudaSuccess) {
+            const size_t w = static_cast<size_t>(tn) * H * cfg->d_v * eo;
+            e = cudaMemcpy2DAsync(static_cast<unsigned char*>(y) + static_cast<size_t>(t0) * H * cfg->d_v * eo,
+                                  static_cast<size_t>(T) * H * cfg->d_v * eo, base + hp.y_off[buf], w, w,
+                                  static_cast<size_t>(B), cudaMemcpyDeviceToHost, sout);
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out[buf], sout);
+    }
+    // the caller's stream ends after the last copy out
+    if (e == cudaSuccess && st == RAMNET_OK) {
+        for (int b2 = 0; b2 < 2 && e == cudaSuccess; ++b2) e = cudaStreamWaitEvent(s, ev_out[b2], 0);
+        for (int b2 = 0; b2 < 2 && e == cudaSuccess; ++b2) e = cudaStreamWaitEvent(s, ev_in[b2], 0);
+    }
+    // streams and events are released once their work is done
+    if (sin) cudaStreamDestroy(sin);
+    if (sout) cudaStreamDestroy(sout);
+    if (ev_start) cudaEventDestroy(ev_start);
+    for (int i = 0; i < 2; ++i) {
+        if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+        if (ev_done[i]) cudaEventDestroy(ev_done[i]);
+        if (ev_out[i]) cudaEventDestroy(ev_out[i]);
+    }
+    if (st != RAMNET_OK) return st;
+    if (e != cudaSuccess) return cuda_fail(e, "scan from host: copies and ordering");
     return RAMNET_OK;
 }
 

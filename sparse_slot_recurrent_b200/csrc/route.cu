@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kRouteThreads, KMAX == 32 ? 3 : 1) k_route(Rou
         const bool cape = p.cape_mask != nullptr && p.cape_mask[h] != 0;
         int32_t pm = 0;
         if (cape) {
-            const int64_t pos = static_cast<int64_t>(p.pos0 != nullptr ? p.pos0[b] : 0) + t;
+            const int64_t pos = static_cast<int64_t>(p.pos0 != nullptr ? p.pos0[b] : 0) + p.t_offset + t;
             int64_t r = pos % p.M;
             pm = static_cast<int32_t>(r < 0 ? r + p.M : r);
         }

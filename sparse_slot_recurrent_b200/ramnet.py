@@ -25,6 +25,7 @@ RAMNET_F32, RAMNET_BF16 = 0, 1
 # every symbol include/ramnet.h declares
 EXPORTED = ("ramnet_decode_addresses", "ramnet_scan_workspace_bytes", "ramnet_scan_layout", "ramnet_scan_forward",
             "ramnet_scan_route", "ramnet_scan_recur", "ramnet_scan_forward_noalloc", "ramnet_decode_step",
+            "ramnet_scan_forward_host_scratch_bytes", "ramnet_scan_forward_host",
             "ramnet_selftest_wait_timeout", "ramnet_set_scan_wait_limit", "ramnet_sync_status", "ramnet_last_error")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # RAMNET_NOALLOC_SCRATCH_BYTES
 
@@ -108,6 +109,11 @@ def load() -> ctypes.CDLL:
                                        ctypes.c_int, _P]
     lib.ramnet_selftest_wait_timeout.restype = ctypes.c_int
     lib.ramnet_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
+    lib.ramnet_scan_forward_host_scratch_bytes.restype = ctypes.c_size_t
+    lib.ramnet_scan_forward_host_scratch_bytes.argtypes = [_P, _I, _I, _I, _I, _I, _I]
+    lib.ramnet_scan_forward_host.restype = ctypes.c_int
+    lib.ramnet_scan_forward_host.argtypes = ([_P, _I, _I, _I, _I] + [_P] * 11 + [_I] + [_P] * 2 +
+                                             [_I, _P, ctypes.c_size_t, _P])
     lib.ramnet_set_scan_wait_limit.restype = ctypes.c_int
     lib.ramnet_set_scan_wait_limit.argtypes = [ctypes.c_uint32]
     lib.ramnet_sync_status.restype = ctypes.c_int
@@ -216,6 +222,34 @@ def scan_forward(cfg: Config, k_logits, q_logits, v, g, z, norm_w=None, cape_mas
         ctypes.byref(c), B, T, H, _dt(k_logits), _ptr(k_logits), _ptr(q_logits), _ptr(v), _ptr(g), _ptr(z),
         _ptr(norm_w), _ptr(cape_mask), _ptr(pos0), _ptr(S_in), _ptr(m_in), _ptr(y), _dt(y), _ptr(S_out),
         _ptr(m_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y, S_out, m_out
+
+
+def scan_forward_host_scratch_bytes(cfg: Config, B: int, T: int, H: int, in_dtype, out_dtype, pieces: int) -> int:
+    c = cfg._c()
+    codes = {torch.bfloat16: RAMNET_BF16, torch.float32: RAMNET_F32}
+    n = load().ramnet_scan_forward_host_scratch_bytes(ctypes.byref(c), B, T, H, codes[in_dtype], codes[out_dtype],
+                                                      pieces)
+    if n == 0:
+        raise RamnetError(RAMNET_ERR_INVALID_ARG, last_error() or "bad sizes")
+    return n
+
+
+def scan_forward_host(cfg: Config, k_logits, q_logits, v, g, z, y, S_out, m_out, scratch, pieces=4, norm_w=None,
+                      cape_mask=None, pos0=None, S_in=None, m_in=None, stream=None):
+    """Prefill scan with k_logits, q_logits, v, g, z and y in host memory (CPU tensors, page-locked
+    for overlap) and the rest on the device; run in ``pieces`` runs along T whose copies overlap
+    the kernels.  ``scratch`` is a uint8 device tensor of scan_forward_host_scratch_bytes()."""
+    B, T, H, L = k_logits.shape
+    for t in (k_logits, q_logits, v, g, z, y):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    _dense(norm_w, cape_mask, pos0, S_in, m_in, S_out, m_out, scratch)
+    c = cfg._c()
+    _check(load().ramnet_scan_forward_host(
+        ctypes.byref(c), B, T, H, _dt(k_logits), k_logits.data_ptr(), q_logits.data_ptr(), v.data_ptr(), g.data_ptr(),
+        z.data_ptr(), _ptr(norm_w), _ptr(cape_mask), _ptr(pos0), _ptr(S_in), _ptr(m_in), y.data_ptr(), _dt(y),
+        _ptr(S_out), _ptr(m_out), pieces, _ptr(scratch), scratch.numel() * scratch.element_size(), _stream(stream)))
     return y, S_out, m_out
 
 

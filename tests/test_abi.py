@@ -175,3 +175,26 @@ def test_two_launch_form_checks(lib):
     assert recur(v=None) == ramnet.RAMNET_ERR_INVALID_ARG and "v" in ramnet.last_error()
     assert recur(od=5) == ramnet.RAMNET_ERR_INVALID_ARG
     assert recur(ws=None) == ramnet.RAMNET_ERR_INVALID_ARG
+
+
+def test_scan_from_host_checks(lib):
+    cfg = _cfg()
+    c = cfg._c()
+    B, T, H = 2, 40, 2
+    need = lib.ramnet_scan_forward_host_scratch_bytes(ctypes.byref(c), B, T, H, ramnet.RAMNET_BF16,
+                                                      ramnet.RAMNET_BF16, 3)
+    assert need > lib.ramnet_scan_workspace_bytes(ctypes.byref(c), B, (T + 2) // 3, H)
+    assert lib.ramnet_scan_forward_host_scratch_bytes(ctypes.byref(c), B, T, H, 7, ramnet.RAMNET_BF16, 3) == 0
+
+    def call(pieces=3, scratch_bytes=need, k=FAKE, y=FAKE, scratch=FAKE):
+        return lib.ramnet_scan_forward_host(ctypes.byref(c), B, T, H, ramnet.RAMNET_BF16, k, FAKE, FAKE, FAKE, FAKE,
+                                            None, None, None, None, None, y, ramnet.RAMNET_BF16, FAKE, FAKE, pieces,
+                                            scratch, scratch_bytes, None)
+
+    assert call(pieces=0) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert "pieces" in ramnet.last_error()
+    assert call(scratch_bytes=need - 1) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert "scratch" in ramnet.last_error()
+    assert call(k=None) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert call(y=None) == ramnet.RAMNET_ERR_INVALID_ARG
+    assert call(scratch=FAKE + 4) == ramnet.RAMNET_ERR_INVALID_ARG

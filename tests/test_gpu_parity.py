@@ -571,6 +571,32 @@ def test_scan_full_size_is_deterministic():
         assert torch.equal(a, b2)
 
 
+@pytest.mark.parametrize("pieces", [1, 3, 7])
+def test_scan_from_host_equals_device_scan(pieces):
+    """ramnet_scan_forward_host (inputs and y in page-locked host memory, runs along T with the
+    state carried and copies overlapping the kernels) gives exactly the device scan's y, S, m."""
+    w, inp = _small_inputs(4, 5, 8, 128, 2, 301, 3, torch.bfloat16, "mixed", seed=21)
+    cfg, _ = _cfgs(w)
+    g = torch.Generator().manual_seed(5)
+    S_in = torch.randn((2, 3, w.M, 128), generator=g).cuda()
+    m_in = (torch.rand((2, 3, w.M), generator=g) * 2).cuda()
+    d = _cuda(inp)
+    y, S, m = ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"], cape_mask=d["cape_mask"],
+                                  pos0=d["pos0"], S_in=S_in, m_in=m_in, out_dtype=torch.bfloat16)
+    host = {k: inp[k].contiguous().pin_memory() for k in ("k_logits", "q_logits", "v", "g", "z")}
+    yh = torch.empty(tuple(y.shape), dtype=torch.bfloat16).pin_memory()
+    S2 = torch.empty_like(S)
+    m2 = torch.empty_like(m)
+    scratch = torch.empty(ramnet.scan_forward_host_scratch_bytes(cfg, 2, 301, 3, torch.bfloat16, torch.bfloat16,
+                                                                 pieces), dtype=torch.uint8, device="cuda")
+    ramnet.scan_forward_host(cfg, host["k_logits"], host["q_logits"], host["v"], host["g"], host["z"], yh, S2, m2,
+                             scratch, pieces=pieces, cape_mask=d["cape_mask"], pos0=d["pos0"], S_in=S_in, m_in=m_in)
+    torch.cuda.synchronize()
+    ramnet.sync_status()
+    assert torch.equal(yh, y.cpu())
+    assert torch.equal(S2, S) and torch.equal(m2, m)
+
+
 # ------------------------------------------------------------------ decode step
 
 def _decode_inputs(w: Workload, seed):
