@@ -50,7 +50,7 @@ from sparse_slot_recurrent_b200.workloads import WORKLOADS, generate  # noqa: E4
 METRIC = "RAM-Net layer tokens/s (prefill scan, decode step) and % of HBM roofline"
 # the largest prefill configuration is the headline; the other two are timed beside it
 PREFILL = "prefill_1p3b_top16"
-E2E_PIECES = 8  # runs along T of the end-to-end call (copies of one run overlap another's kernels)
+E2E_PIECES = 16  # runs along T of the end-to-end call (copies of one run overlap another's kernels)
 PREFILL_ALL = ("prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16")
 LAUNCHES_PER_STEP = 2  # route (k_route) and recurrence (k_scan)
 SM_COUNT = 148

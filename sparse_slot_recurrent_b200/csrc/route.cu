@@ -34,9 +34,10 @@ __host__ __device__ inline size_t route_kept_offset(int O, int nchb)
 }
 
 // At K = 32 the search's kept list and merge buffers want ~200 registers; capping them for 3
-// CTAs per SM (a little spilling) is faster than 2 CTAs per SM.
+// CTAs per SM (a little spilling) is faster than 2 CTAs per SM.  At K = 16 the cap keeps 4
+// CTAs per SM (128 registers).
 template <int KMAX, int DPMAX>
-__global__ void __launch_bounds__(kRouteThreads, KMAX == 32 ? 3 : 1) k_route(RouteParams p)
+__global__ void __launch_bounds__(kRouteThreads, KMAX == 32 ? 3 : (KMAX == 16 ? 4 : 1)) k_route(RouteParams p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const int O = p.ncta * p.nw;
