@@ -314,7 +314,9 @@ __device__ __forceinline__ uint64_t merge16(uint64_t a, uint64_t b_rev, int li)
 #pragma unroll
     for (int d = 8; d > 0; d >>= 1) {
         const uint64_t y = __shfl_xor_sync(0xffffffffu, x, d, 16);
-        x = (li & d) ? (x < y ? x : y) : (x > y ? x : y);
+        // the lower lane of a pair keeps the larger word, the upper one the smaller
+        const bool take = (y > x) != ((li & d) != 0);
+        x = take ? y : x;
     }
     return x;
 }
