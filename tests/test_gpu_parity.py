@@ -666,6 +666,46 @@ def test_decode_step_cooperative_search_matches_oracle(d_p, U, K, mode, renorm):
     assert _maxabs(S, oS) <= TOL_F32 and _maxabs(m, om) <= TOL_F32
 
 
+STEP_PERSISTENT_CASES = [
+    # d_p, U, K, logit mode, renorm, d_v -- shapes served by the persistent decode-step kernel
+    (4, 5, 32, "ties", 1, 128),
+    (4, 5, 32, "mixed", 0, 64),
+    (16, 2, 8, "normal", 1, 128),
+    (3, 5, 64, "ties", 1, 32),
+    (16, 3, 20, "mixed", 1, 16),
+]
+
+
+@pytest.mark.parametrize("d_p,U,K,mode,renorm,d_v", STEP_PERSISTENT_CASES)
+def test_decode_step_persistent_kernel_matches_oracle(d_p, U, K, mode, renorm, d_v):
+    """Decode steps with K > 16 or d_p > 8, which run the persistent kernel (decoder warps with
+    the one-thread search, row warps per unit), against the oracle over three steps."""
+    B, H, steps = 3, 4, 3
+    cfg = ramnet.Config(d_p=d_p, U=U, K=K, d_v=d_v, renorm=renorm)
+    ocfg = oracle.OracleConfig(d_p=d_p, U=U, K=K, d_v=d_v, renorm=renorm)
+    M = d_p ** U
+    g = torch.Generator().manual_seed(d_p * 100 + K)
+    S0 = torch.randn((B, H, M, d_v), generator=g)
+    m0 = torch.rand((B, H, M), generator=g) + 0.5
+    S, m = S0.cuda(), m0.cuda()
+    oS, om = S0.double().numpy().copy(), m0.double().numpy().copy()
+    mask = torch.tensor([1, 1, 0, 1], dtype=torch.uint8)
+    kl = _logits(B, steps, H, d_p * U, mode, torch.bfloat16, seed=K + 3)
+    ql = _logits(B, steps, H, d_p * U, mode, torch.bfloat16, seed=K + 4)
+    for t in range(steps):
+        v = torch.randn((B, H, d_v), generator=g).to(torch.bfloat16)
+        z = torch.sigmoid(torch.randn((B, H, d_v), generator=g)).to(torch.bfloat16)
+        gt = torch.sigmoid(torch.randn((B, H), generator=g)).to(torch.bfloat16)
+        pos = torch.tensor([t, 9 + t, 2 * M + t], dtype=torch.int32)
+        k_t, q_t = kl[:, t].contiguous(), ql[:, t].contiguous()
+        y = ramnet.decode_step(cfg, k_t.cuda(), q_t.cuda(), v.cuda(), gt.cuda(), z.cuda(), S, m, pos=pos.cuda(),
+                               cape_mask=mask.cuda(), out_dtype=torch.float32)
+        oy = oracle.decode_step(ocfg, k_t, q_t, v, gt, z, oS, om, pos=pos, cape_mask=mask)
+        ramnet.sync_status()
+        assert _maxabs(y, oy) <= TOL_BF16
+    assert _maxabs(S, oS) <= TOL_BF16 and _maxabs(m, om) <= TOL_BF16
+
+
 def test_decode_step_full_size_sampled_units():
     """One step of the full batched decode workload (state resident in HBM); sampled
     (b,h) units are recomputed by the oracle from their pre-step state."""
