@@ -59,6 +59,7 @@ SM_COUNT = 148
 TMEM_BYTES_PER_CLK_SM = 120.0
 DECODE = "decode_b256"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # HBM3e nominal (DGX B200 figure), for context beside the measured peak
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -262,6 +263,39 @@ def cpu_baseline(w, cores: int):
             "seconds": round(secs, 3)}
 
 
+def decode_cpu_baseline(w, cores: int, max_seconds: float = 10.0):
+    """The CPU oracle's decode step on a bounded sample of the decode workload: 8 sequences
+    x H heads, steps until about max_seconds; units split over the host cores (the oracle
+    call releases the interpreter lock)."""
+    import concurrent.futures
+    import numpy as np
+    import oracle
+    oracle.build()
+    sub = w.with_(B=min(w.B, 8))
+    inp = generate(sub, seed=0)
+    gen = torch.Generator().manual_seed(1)
+    S = torch.randn((sub.B, sub.H, sub.M, sub.d_v), generator=gen).double().numpy()
+    m = (torch.rand((sub.B, sub.H, sub.M), generator=gen) * 1.5 + 0.5).double().numpy()
+    ocfg = oracle.OracleConfig(d_p=w.d_p, U=w.U, K=w.K, d_v=w.d_v)
+    units = sub.B * sub.H
+    parts = [(units * i // cores, units * (i + 1) // cores) for i in range(cores)]
+    parts = [pr for pr in parts if pr[1] > pr[0]]
+    steps = 0
+    t0 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(len(parts)) as ex:
+        while steps < sub.T and (time.perf_counter() - t0) < max_seconds:
+            r = steps % sub.ring
+            args = [inp[k][:, r].contiguous() for k in ("k_logits", "q_logits", "v", "g", "z")]
+            pos = torch.full((sub.B,), steps, dtype=torch.int32)
+            list(ex.map(lambda pr: oracle.decode_step(ocfg, *args, S, m, pos=pos, cape_mask=inp["cape_mask"],
+                                                      units=pr), parts))
+            steps += 1
+    secs = time.perf_counter() - t0
+    return {"value": sub.B * steps / secs, "unit": "tokens/s", "cores": len(parts), "kind": "oracle",
+            "sample": f"{sub.B} sequences x {sub.H} heads x {steps} consecutive steps of {w.name}",
+            "seconds": round(secs, 3)}
+
+
 def run_reference(args, world, rank):
     """The reference arm: the CPU oracle, timed on the host cores, rank 0 only."""
     if rank != 0:
@@ -379,7 +413,8 @@ def time_prefill(args, world, rank, local, w, with_e2e: bool):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
                 "kernel": "k_scan (ramnet_scan_recur)", "algorithmic_bytes": alg_recur,
-                "ms_per_launch": recur_ms, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)"}
+                "ms_per_launch": recur_ms, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)",
+                "frac_of_nominal": achieved / NOMINAL_HBM_GBS}
     # on-chip: the slot state the recurrence reads and writes (tensor memory), against the
     # tensor-memory bandwidth measured on this machine at the sampled SM clock
     sm_mhz = clk["sm_mhz"] if clk else 1965.0
@@ -445,6 +480,8 @@ def run_gpu(args, world, rank, local):
     ramnet.load()
     if args.no_prefill:  # decode only (profiler captures of the decode step)
         decode = run_decode(args, world, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            decode["cpu_baseline"] = decode_cpu_baseline(WORKLOADS[DECODE], os.cpu_count() or 1)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "decode": decode}), flush=True)
         return
@@ -467,6 +504,8 @@ def run_gpu(args, world, rank, local):
                 "gpu_launches": main["gpu_launches"], "clocks": main["clocks"], "prefill": prefill, "decode": decode}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(head, os.cpu_count() or 1)
+            if decode is not None:
+                decode["cpu_baseline"] = decode_cpu_baseline(WORKLOADS[DECODE], os.cpu_count() or 1)
         print(json.dumps(line), flush=True)
 
 
@@ -525,8 +564,9 @@ def run_decode(args, world, local):
             "d_v": w.d_v, "value": weak_scaling_value(w.B * w.T, world, ms), "unit": "tokens/s",
             "ms_per_step": step_ms, "gpu_launches_per_replay": w.T,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "k_decode_step",
-                         "algorithmic_bytes_per_step": alg, "peak_kind": f"{peak_kind} hbm_gbs"},
+                         "frac": achieved / peak, "traffic": None, "kernel": "k_step_warp",
+                         "algorithmic_bytes_per_step": alg, "peak_kind": f"{peak_kind} hbm_gbs",
+                         "frac_of_nominal": achieved / NOMINAL_HBM_GBS},
             "l2": "state (8 GiB) larger than L2",
             "state_elements_per_step": state_elements_per_step(w.K, w.d_v, w.B * w.H)}
 
