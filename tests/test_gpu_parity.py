@@ -597,6 +597,28 @@ def test_scan_from_host_equals_device_scan(pieces):
     assert torch.equal(S2, S) and torch.equal(m2, m)
 
 
+def test_scan_from_host_fp32_pageable_equals_device_scan():
+    """ramnet_scan_forward_host with fp32 inputs and output in ordinary (pageable) host memory,
+    no initial state, T not a multiple of the runs: the same bits as the device scan."""
+    w, inp = _small_inputs(4, 4, 16, 64, 2, 157, 2, torch.float32, "all", seed=31)
+    cfg, _ = _cfgs(w)
+    d = _cuda(inp)
+    y, S, m = ramnet.scan_forward(cfg, d["k_logits"], d["q_logits"], d["v"], d["g"], d["z"], cape_mask=d["cape_mask"],
+                                  pos0=d["pos0"], out_dtype=torch.float32)
+    host = {k: inp[k].contiguous() for k in ("k_logits", "q_logits", "v", "g", "z")}
+    yh = torch.empty(tuple(y.shape), dtype=torch.float32)
+    S2 = torch.empty_like(S)
+    m2 = torch.empty_like(m)
+    scratch = torch.empty(ramnet.scan_forward_host_scratch_bytes(cfg, 2, 157, 2, torch.float32, torch.float32, 5),
+                          dtype=torch.uint8, device="cuda")
+    ramnet.scan_forward_host(cfg, host["k_logits"], host["q_logits"], host["v"], host["g"], host["z"], yh, S2, m2,
+                             scratch, pieces=5, cape_mask=d["cape_mask"], pos0=d["pos0"])
+    torch.cuda.synchronize()
+    ramnet.sync_status()
+    assert torch.equal(yh, y.cpu())
+    assert torch.equal(S2, S) and torch.equal(m2, m)
+
+
 # ------------------------------------------------------------------ decode step
 
 def _decode_inputs(w: Workload, seed):
