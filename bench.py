@@ -55,7 +55,7 @@ PREFILL_ALL = ("prefill_340m_top8", "prefill_340m_top32", "prefill_1p3b_top16")
 LAUNCHES_PER_STEP = 2  # route (k_route) and recurrence (k_scan)
 SM_COUNT = 148
 # tensor-memory bytes per clock per SM (32x32b.x4 load and store, many warps, batched waits),
-# measured on this machine; the on-chip roofline denominator
+# measured with a tcgen05.ld/st probe on B200; the on-chip roofline denominator
 TMEM_BYTES_PER_CLK_SM = 120.0
 DECODE = "decode_b256"
 FALLBACK_HBM_GBS = 6650.0
@@ -416,7 +416,7 @@ def time_prefill(args, world, rank, local, w, with_e2e: bool):
                 "ms_per_launch": recur_ms, "peak_kind": f"{peak_kind} hbm_gbs (burst copy)",
                 "frac_of_nominal": achieved / NOMINAL_HBM_GBS}
     # on-chip: the slot state the recurrence reads and writes (tensor memory), against the
-    # tensor-memory bandwidth measured on this machine at the sampled SM clock
+    # tensor-memory bandwidth of a tcgen05.ld/st probe (TMEM_BYTES_PER_CLK_SM) at the sampled SM clock
     sm_mhz = clk["sm_mhz"] if clk else 1965.0
     ctas = w.B * w.H * lay.ncta
     onchip_peak = TMEM_BYTES_PER_CLK_SM * min(ctas, SM_COUNT) * sm_mhz * 1e6 / 1e9
